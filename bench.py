@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of one MoE routing pass per step on B200.
+
+A step is the whole hot path over one batch: router top-K gating, the padded
+expert layout (histogram + scan), the dispatch scatter (FP8 e4m3 with
+128-channel scales for the default workload) and the combine with the FarSkip
+dual-residual epilogue, all through the C ABI on one stream.  The expert GEMMs
+are not part of the path: their outputs y are a resident synthetic buffer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Default workload: the DeepSeek-V3-shaped
+prefill (S=4096 tokens, H=7168, E=256, K=8, R=8, FP8 dispatch, dual-residual
+combine).  Its per-step working set (~1.5 GB) is far larger than L2, so no
+L2 flush is needed between steps.  With N > 1 (torchrun) each rank runs an
+independent replica on its own GPU (no data-path collective); timing is the
+max over ranks.
+
+--impl reference times the CPU oracle (test infrastructure, plain C,
+single-threaded) on this machine's host cores over a bounded sample of the
+same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------------------------
+# workload accounting
+# ----------------------------------------------------------------------------------------------
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes each step must move at least (padding rows and dense E-wide work excluded)."""
+    b = w.esize
+    bout = 1 if w.quant == "fp8" else b
+    S, H, E, K = w.S, w.H, w.E, w.K
+    route = S * E * 4 + S * K * 8
+    layout = S * K * 4 * 3 + E * 8
+    dispatch = S * H * b + S * K * H * bout + S * K * 4
+    if w.quant == "fp8":
+        dispatch += S * K * (H // 128) * 4
+    combine = S * K * H * b + S * K * 8 + (4 * S * H * b if w.fused else S * H * b)
+    return dict(route=route, layout=layout, dispatch=dispatch, combine=combine)
+
+
+def workload_config(w, world: int) -> dict:
+    return {
+        "workload": w.name, "tokens_per_gpu": w.S, "S": w.S, "H": w.H, "E": w.E, "K": w.K,
+        "R_logical_ranks": w.R, "token_padding": w.P,
+        "activations": w.dtype, "dispatch": "fp8_e4m3_block128" if w.quant == "fp8" else w.dtype,
+        "combine": "dual_residual" if w.fused else "plain", "accumulate": "fp32",
+        "global_batch": w.S * world, "parallelism": f"replicas x{world}",
+        "l2": "no flush: per-step working set >> 126 MB L2",
+    }
+
+
+def read_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged.
+
+    A summary under profiles/ carries lines 'kernel_source_sha256: <hex>',
+    'workload: <name>' and 'dram_bytes_per_launch: <int>'."""
+    src = os.path.join(ROOT, "combine_moe_route_09_b200", "csrc", kernel_file)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        kv = {}
+        for line in open(os.path.join(pdir, fn)):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip().strip("-* `")] = v.strip().strip("`")
+        if kv.get("kernel_source_sha256") == sha and kv.get("workload") == workload \
+                and "dram_bytes_per_launch" in kv:
+            try:
+                return int(kv["dram_bytes_per_launch"])
+            except ValueError:
+                return None
+    return None
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ----------------------------------------------------------------------------------------------
+
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.idx, self.period = device_index, period_s
+        self.samples, self.reasons, self.max_mhz, self.err = [], 0, None, None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _poll(self, nv, h):
+        self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+
+    def _run(self):
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._poll(nv, h)
+            while not self._stop.wait(self.period):
+                self._poll(nv, h)
+            self._poll(nv, h)
+            nv.nvmlShutdown()
+        except Exception as e:  # clocks are reported as unavailable, the run goes on
+            self.err = repr(e)
+
+    def start(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        time.sleep(0.02)
+
+    def stop(self) -> dict:
+        self._stop.set()
+        self._t.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "error": self.err}
+        names = [n for bit, n in _REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle baseline (test infrastructure; this leg alone may run it)
+# ----------------------------------------------------------------------------------------------
+
+def oracle_pass(w, inp: dict, S: int):
+    import oracle
+
+    lg = inp["logits"][:S]
+    idx, wt = oracle.route_topk(lg, w.K)
+    lay = oracle.layout(idx, w.E, w.R, w.P)
+    q = oracle.QUANT_FP8_E4M3_B128 if w.quant == "fp8" else oracle.QUANT_NONE
+    oracle.dispatch(inp["x"][:S], lay["slot_of"], lay["cap"], quant=q)
+    y = inp["y"][:lay["cap"]]
+    oracle.combine(y, lay["slot_of"], wt, inp["shared"][:S] if w.fused else None,
+                   inp["residual"][:S] if w.fused else None)
+
+
+def cpu_baseline(w, inp: dict, min_seconds: float = 10.0) -> dict:
+    """Full workload through the oracle, repeated until min_seconds of CPU work."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_pass(w, inp, w.S)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": w.S * n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} full pass(es) of {w.name} (S={w.S}) through the single-threaded C oracle, "
+                      f"{el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------------------------
+
+def host_inputs(w) -> dict:
+    from combine_moe_route_09_b200 import synth
+
+    d = dict(logits=synth.logits(w), x=synth.activations(w), y=synth.expert_outputs(w))
+    if w.fused:
+        d["shared"], d["residual"] = synth.shared_out(w), synth.residual(w)
+    return d
+
+
+def run_reference(args, w, world):
+    """CPU oracle as the reference arm: rank 0 only, a bounded token sample per step."""
+    inp = host_inputs(w)
+    n_cal = min(w.S, 256)
+    t0 = time.perf_counter()
+    oracle_pass(w, inp, n_cal)
+    per_tok = (time.perf_counter() - t0) / n_cal
+    budget = 60.0  # seconds for warm-up + timed steps together
+    S_sample = int(max(1, min(w.S, budget / max(1, args.steps + args.warmup) / per_tok)))
+    for _ in range(args.warmup):
+        oracle_pass(w, inp, S_sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(w, inp, S_sample)
+    el = time.perf_counter() - t0
+    value = S_sample * args.steps / el
+    sample = (f"first {S_sample} of {w.S} tokens of {w.name} per step (same H, E, K, R, padding, "
+              f"quantisation and epilogue), single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded)", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": 1,
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+
+    from combine_moe_route_09_b200 import synth
+    from combine_moe_route_09_b200.buffer import MoeBuffer
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    inp = host_inputs(w)
+    pinned = {k: synth.to_torch(v).pin_memory() for k, v in inp.items()}
+    d = {k: v.to(device, non_blocking=True) for k, v in pinned.items()}
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device)
+    sh, rs = (d["shared"], d["residual"]) if w.fused else (None, None)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        buf.step(d["logits"], d["x"], d["y"], sh, rs)
+    torch.cuda.synchronize()
+    if buf.read_status() != 0:
+        raise RuntimeError("device status flagged a problem during warm-up")
+
+    # ---- device-timed region: K steps, CUDA events on the launching stream ----
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(K):
+        e = ev[i]
+        e[0].record()
+        buf.route(d["logits"])
+        e[1].record()
+        buf.plan()
+        e[2].record()
+        buf.dispatch(d["x"])
+        e[3].record()
+        buf.combine(d["y"], sh, rs)
+        e[4].record()
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, device)
+    phase_names = ["route", "layout", "dispatch", "combine"]
+    phase_ms = {p: statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
+                for j, p in enumerate(phase_names)}
+    status = buf.read_status()
+    counts_ok = int(buf.layout.counts.sum().item()) == w.S * w.K
+    if status != 0 or not counts_ok:
+        raise RuntimeError(f"bench sanity check failed: status={status} counts_ok={counts_ok}")
+
+    # ---- end to end: pinned host inputs in, both residual streams out, every step ----
+    e2e = None
+    if not args.no_e2e:
+        Ke = min(K, args.e2e_steps)
+        out_h = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+        rnr_h = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory() if w.fused else None
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = out_h.numel() * out_h.element_size() * (2 if w.fused else 1)
+
+        def e2e_step():
+            for k, v in pinned.items():
+                d[k].copy_(v, non_blocking=True)
+            buf.step(d["logits"], d["x"], d["y"], sh, rs)
+            out_h.copy_(buf.out, non_blocking=True)
+            if rnr_h is not None:
+                rnr_h.copy_(buf.out_no_routed, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(Ke):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
+        e2e = {"value": w.S * world * Ke / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+               "ms_per_step": e2e_ms / Ke,
+               "path": "MoeBuffer.step via the C ABI; pinned host inputs copied in and both residual "
+                       "streams copied out each step, inside the timed region"}
+
+    if rank != 0:
+        return
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = read_peak_hbm()
+    phases = {}
+    for p in phase_names:
+        gbs = ab[p] / (phase_ms[p] * 1e-3) / 1e9
+        phases[p] = {"us": phase_ms[p] * 1e3, "algorithmic_bytes": ab[p], "gb_s": gbs,
+                     "frac_of_peak": gbs / peak}
+    dc_ms = phase_ms["dispatch"] + phase_ms["combine"]
+    dc_gbs = (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3) / 1e9
+    comb = phases["combine"]
+    roofline = {"kernel": "combine_kernel (gather + weighted sum + dual residual)", "bound": "hbm",
+                "achieved": comb["gb_s"], "peak": peak, "unit": "GB/s", "frac": comb["gb_s"] / peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_launch": ab["combine"],
+                "traffic": recorded_traffic("combine.cu", w.name)}
+    line = {
+        "metric": METRIC, "value": w.S * world * K / (total_ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; no dataset or weights)", "config": workload_config(w, world),
+        "dispatch_combine": {"tokens_per_s": w.S * world / (dc_ms * 1e-3), "effective_gb_s": dc_gbs,
+                             "frac_of_peak": dc_gbs / peak, "frac_of_nominal_8tbs": dc_gbs / 8000.0},
+        "phases": phases, "roofline": roofline, "e2e": e2e,
+        "gpu_launches": K * buf.KERNELS_PER_STEP, "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp)
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="4", help="1, 2, 2b, 3, 4 or 5 (default 4)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from combine_moe_route_09_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+"""Thin Python binding over the C ABI in ``include/moe_route.h``.
+
+Argument marshalling only: each function checks tensor dtypes/devices,
+allocates outputs the caller did not pass, and calls the C entry point of the
+same name on the current CUDA stream.  All arithmetic runs in the CUDA kernels
+of ``libmoe_route.so``; there is no CPU fallback, and a missing or unloadable
+library raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_route.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA = 0, 1, 2
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+MOE_QUANT_NONE, MOE_QUANT_FP8_E4M3_B128 = 0, 1
+MOE_STATUS_BAD_INDEX, MOE_STATUS_OVERFLOW, MOE_STATUS_BAD_SLOT = 1, 2, 4
+MOE_MAX_EXPERTS, MOE_MAX_TOPK = 1024, 32
+
+_P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+# name -> (restype, argtypes), the exact C signatures
+SIGNATURES = {
+    "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
+    "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _Z, _P, _P]),
+    "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
+    "moe_combine_dual_residual": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_error_string": (ctypes.c_char_p, [_I]),
+    "moe_capacity": (_L, [_I, _I, _I, _I]),
+}
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, rc: int):
+        msg = lib().moe_error_string(rc).decode()
+        super().__init__(f"{fn} failed: {msg} (code {rc})")
+        self.rc = rc
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe_route.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library missing: {LIB_PATH}; build it with "
+                               "`python -m combine_moe_route_09_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def _dev(t: torch.Tensor, name: str, dtypes, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    return t
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return MOE_DTYPE_F32 if t.dtype == torch.float32 else MOE_DTYPE_BF16
+
+
+_ACT = (torch.float32, torch.bfloat16)
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
+
+
+def moe_capacity(S: int, E: int, K: int, token_padding: int) -> int:
+    return int(lib().moe_capacity(S, E, K, token_padding))
+
+
+def moe_route_topk(logits: torch.Tensor, K: int, topk_idx=None, topk_w=None, stream=None):
+    """Top-K experts per token (descending logit, ties to the lower id) and softmax weights."""
+    _dev(logits, "logits", (torch.float32,))
+    S, E = logits.shape
+    if topk_idx is None:
+        topk_idx = torch.empty((S, K), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((S, K), dtype=torch.float32, device=logits.device)
+    _dev(topk_idx, "topk_idx", (torch.int32,), (S, K))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    _check("moe_route_topk", lib().moe_route_topk(_ptr(logits), S, E, K, _ptr(topk_idx), _ptr(topk_w),
+                                                   _stream(stream, logits.device)))
+    return topk_idx, topk_w
+
+
+def moe_dispatch_layout_workspace(S: int, E: int, K: int) -> int:
+    return int(lib().moe_dispatch_layout_workspace(S, E, K))
+
+
+class Layout(NamedTuple):
+    counts: torch.Tensor        # [E]    tokens_per_expert
+    offsets: torch.Tensor       # [E+1]  cu_seqlens of the padded groups
+    rank_offsets: torch.Tensor  # [R+1]
+    slot_of: torch.Tensor       # [S,K]
+    row_src: torch.Tensor       # [cap]
+    cap: int
+
+
+def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, token_padding: int = 0,
+                        cap: Optional[int] = None, *, workspace=None, status=None, out=None,
+                        stream=None) -> Layout:
+    """Histogram + prefix scan into the padded expert-contiguous layout.
+
+    ``workspace`` (uint8, >= moe_dispatch_layout_workspace bytes) must be zero-filled
+    before its first use; each call leaves it zeroed.  A fresh zeroed one is
+    allocated when it is not given.  ``out`` may carry a Layout to write into."""
+    _dev(topk_idx, "topk_idx", (torch.int32,))
+    S, K = topk_idx.shape
+    dev = topk_idx.device
+    if cap is None:
+        cap = moe_capacity(S, E, K, token_padding)
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                     torch.empty((S, K), **i32), torch.empty(max(cap, 0), **i32), cap)
+    need = moe_dispatch_layout_workspace(S, E, K)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", (torch.uint8,))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_dispatch_layout", lib().moe_dispatch_layout(
+        _ptr(topk_idx), S, E, K, R, token_padding, _ptr(out.counts), _ptr(out.offsets),
+        _ptr(out.rank_offsets), _ptr(out.slot_of), _ptr(out.row_src), cap, _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream, dev)))
+    return out._replace(cap=cap)
+
+
+def moe_dispatch(x: torch.Tensor, slot_of: torch.Tensor, cap: int, quant: int = MOE_QUANT_NONE,
+                 xd=None, xs=None, status=None, stream=None):
+    """Scatter rows of x [S,H] into xd [cap,H]; with FP8 also scales xs [cap,H/128]."""
+    _dev(x, "x", _ACT)
+    S, H = x.shape
+    K = slot_of.shape[1]
+    _dev(slot_of, "slot_of", (torch.int32,), (S, K))
+    if quant == MOE_QUANT_FP8_E4M3_B128:
+        if xd is None:
+            xd = torch.empty((cap, H), dtype=torch.float8_e4m3fn, device=x.device)
+        if xs is None:
+            xs = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+        _dev(xd, "xd", _FP8, (cap, H))
+        _dev(xs, "xs", (torch.float32,), (cap, H // 128))
+    else:
+        if xd is None:
+            xd = torch.empty((cap, H), dtype=x.dtype, device=x.device)
+        _dev(xd, "xd", (x.dtype,), (cap, H))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_dispatch", lib().moe_dispatch(_ptr(x), _dtype_code(x), S, H, K, _ptr(slot_of), quant,
+                                               _ptr(xd), _ptr(xs), cap, _ptr(status),
+                                               _stream(stream, x.device)))
+    return xd, xs
+
+
+def moe_combine_dual_residual(y: torch.Tensor, slot_of: torch.Tensor, topk_w: torch.Tensor,
+                              shared_out=None, residual=None, residual_out=None,
+                              residual_no_routed_out=None, want_no_routed: bool = True,
+                              status=None, stream=None):
+    """Weighted gather back to token order with the FarSkip dual-residual epilogue.
+
+    Returns (residual_out, residual_no_routed_out); the second is None unless both
+    shared_out and residual are given (and want_no_routed)."""
+    _dev(y, "y", _ACT)
+    cap, H = y.shape
+    S, K = slot_of.shape
+    _dev(slot_of, "slot_of", (torch.int32,))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    for name, t in (("shared_out", shared_out), ("residual", residual)):
+        if t is not None:
+            _dev(t, name, (y.dtype,), (S, H))
+    if residual_out is None:
+        residual_out = torch.empty((S, H), dtype=y.dtype, device=y.device)
+    _dev(residual_out, "residual_out", (y.dtype,), (S, H))
+    if residual_no_routed_out is None and want_no_routed and shared_out is not None \
+            and residual is not None:
+        residual_no_routed_out = torch.empty((S, H), dtype=y.dtype, device=y.device)
+    if residual_no_routed_out is not None:
+        _dev(residual_no_routed_out, "residual_no_routed_out", (y.dtype,), (S, H))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_combine_dual_residual", lib().moe_combine_dual_residual(
+        _ptr(y), _dtype_code(y), S, H, K, cap, _ptr(slot_of), _ptr(topk_w), _ptr(shared_out),
+        _ptr(residual), _ptr(residual_out), _ptr(residual_no_routed_out), _ptr(status),
+        _stream(stream, y.device)))
+    return residual_out, residual_no_routed_out

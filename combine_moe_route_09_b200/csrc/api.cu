@@ -1,0 +1,128 @@
+// C-ABI entry points: host-side argument checks, then the launches.  Every
+// entry point only enqueues work on the caller's stream.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "moe_route.h"
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int current_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+int esize(int dtype) { return dtype == MOE_DTYPE_F32 ? 4 : (dtype == MOE_DTYPE_BF16 ? 2 : 0); }
+
+int to_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Activation rows: 16-byte aligned base and a row size that is a multiple of 16 bytes.
+bool rows_ok(const void *p, int H, int bytes_per_elem) {
+    return p && aligned(p, 16) && ((size_t)H * bytes_per_elem) % 16 == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_error_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA launch error";
+        default: return "unknown error";
+    }
+}
+
+int64_t moe_capacity(int S, int E, int K, int token_padding) {
+    if (S < 0 || E < 1 || K < 1 || token_padding < 0) return -1;
+    return (int64_t)S * K + (int64_t)E * (token_padding > 0 ? token_padding - 1 : 0);
+}
+
+int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, float *topk_w,
+                   void *stream) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > E || K > MOE_MAX_TOPK)
+        return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_route_topk(logits, S, E, K, topk_idx, topk_w,
+                                        static_cast<cudaStream_t>(stream), current_sms()));
+}
+
+size_t moe_dispatch_layout_workspace(int S, int E, int K) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK) return 0;
+    if ((int64_t)S * K >= ((int64_t)1 << 31)) return 0;
+    return moe::layout_workspace_bytes(S, E, K);
+}
+
+int moe_dispatch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int token_padding,
+                        int32_t *counts, int32_t *offsets, int32_t *rank_offsets, int32_t *slot_of,
+                        int32_t *row_src, int64_t cap, void *workspace, size_t workspace_bytes,
+                        int32_t *status, void *stream) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK || R < 1 || E % R != 0 ||
+        token_padding < 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    // The padded layout must be addressable with int32 rows whatever the routing.
+    if ((int64_t)S * K + (int64_t)E * (token_padding > 0 ? token_padding - 1 : 0) >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !rank_offsets || !workspace) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!topk_idx || !slot_of)) return MOE_ERR_INVALID_ARG;
+    if (cap > 0 && !row_src) return MOE_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || workspace_bytes < moe::layout_workspace_bytes(S, E, K))
+        return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {topk_idx, counts, offsets, rank_offsets, slot_of, row_src, status};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_layout(topk_idx, S, E, K, R, token_padding, counts, offsets,
+                                    rank_offsets, slot_of, row_src, cap, workspace, status,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int moe_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
+                 void *xd, float *xs, int64_t cap, int32_t *status, void *stream) {
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (quant != MOE_QUANT_NONE && quant != MOE_QUANT_FP8_E4M3_B128) return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!slot_of || !aligned(slot_of, 4) || (status && !aligned(status, 4))) return MOE_ERR_INVALID_ARG;
+    if (!rows_ok(x, H, b)) return MOE_ERR_INVALID_ARG;
+    if (quant == MOE_QUANT_NONE) {
+        if (xs || (cap > 0 && !rows_ok(xd, H, b))) return MOE_ERR_INVALID_ARG;
+    } else {
+        if (H % 128 != 0 || (cap > 0 && (!rows_ok(xd, H, 1) || !xs || !aligned(xs, 4))))
+            return MOE_ERR_INVALID_ARG;
+    }
+    if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_dispatch(x, dtype, S, H, K, slot_of, quant, xd, xs, cap, status,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int64_t cap,
+                              const int32_t *slot_of, const float *topk_w, const void *shared_out,
+                              const void *residual, void *residual_out,
+                              void *residual_no_routed_out, int32_t *status, void *stream) {
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (residual_no_routed_out && !(shared_out && residual)) return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!slot_of || !topk_w || !aligned(slot_of, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+    if (status && !aligned(status, 4)) return MOE_ERR_INVALID_ARG;
+    if ((cap > 0 && !rows_ok(y, H, b)) || !rows_ok(residual_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if (shared_out && !rows_ok(shared_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if (residual && !rows_ok(residual, H, b)) return MOE_ERR_INVALID_ARG;
+    if (residual_no_routed_out && !rows_ok(residual_no_routed_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_combine(y, dtype, S, H, K, cap, slot_of, topk_w, shared_out, residual,
+                                     residual_out, residual_no_routed_out, status,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Layout tiling: a CTA of LT_WARPS warps takes LT_TILE consecutive (token, k)
+// pairs; each warp takes LT_ITEMS consecutive chunks of 32 pairs.
+constexpr int LT_WARPS = 16;
+constexpr int LT_ITEMS = 4;
+constexpr int LT_THREADS = LT_WARPS * 32;
+constexpr int LT_TILE = LT_THREADS * LT_ITEMS;
+constexpr size_t LT_HEADER = 256;
+
+inline int layout_tiles(long long npairs) {
+    long long t = (npairs + LT_TILE - 1) / LT_TILE;
+    return t < 1 ? 1 : (int)t;
+}
+
+inline size_t layout_workspace_bytes(int S, int E, int K) {
+    const size_t hist = (size_t)layout_tiles((long long)S * K) * (size_t)E * 4;
+    return LT_HEADER + ((hist + 255) / 256) * 256;
+}
+
+cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t *idx, float *w,
+                              cudaStream_t st, int sms);
+
+cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int P,
+                          int32_t *counts, int32_t *offsets, int32_t *rank_offsets,
+                          int32_t *slot_of, int32_t *row_src, int64_t cap, void *workspace,
+                          int32_t *status, cudaStream_t st);
+
+cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of,
+                            int quant, void *xd, float *xs, int64_t cap, int32_t *status,
+                            cudaStream_t st);
+
+cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_t cap,
+                           const int32_t *slot_of, const float *topk_w, const void *shared_out,
+                           const void *residual, void *out, void *out_no_routed, int32_t *status,
+                           cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,256 @@
+// Per-expert histogram and prefix scan into the padded, expert-contiguous layout.
+//
+// "MoonEP developer guide", core API example and tuning parameters:
+// tokens_per_expert, cu_seqlens, groups padded to token_padding rows.
+// "Efficient and portable mixture-of-experts communication", Portable Kernels
+// (a fixed receive bound per (rank, local expert); experts in blocks of E/R)
+// and Dispatch (tokens of one expert contiguous; the source of each row kept
+// for the combine).
+//
+// Two kernels, no spin-waits and no global atomics except one arrival counter:
+//
+//  layout_hist   one CTA per tile of LT_TILE pairs.  Each warp ranks its 32
+//                pairs by expert with __match_any_sync (peers share an expert;
+//                the lowest peer adds the group size to the warp's private
+//                shared-memory histogram), so the tile histogram is built
+//                without atomics.  The CTA writes it to hist[tile][E], then
+//                takes a ticket; the CTA with the last ticket (all tiles are
+//                written by then) turns hist into per-expert exclusive prefixes
+//                over tiles, pads the totals and scans them over experts into
+//                counts / offsets / rank_offsets, and resets the ticket.
+//  layout_slots  one CTA per tile again: recomputes the same per-warp ranks,
+//                converts the per-warp histograms to prefixes over warps, and
+//                writes slot = offsets[e] + tile prefix + warp prefix + rank,
+//                then row_src, and -1 into padding rows and rows past offsets[E].
+//
+// The slot of a pair is therefore offsets[e] plus the number of earlier pairs
+// (ascending t*K + k) with the same expert: a stable counting sort.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+struct LayoutHeader {
+    unsigned int ticket;
+};
+
+__device__ __forceinline__ int pad_count(int c, int P) { return P > 0 ? ((c + P - 1) / P) * P : c; }
+
+__global__ void __launch_bounds__(LT_THREADS)
+    layout_hist_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P,
+                       int64_t cap, int32_t *hist, LayoutHeader *hdr, int32_t *__restrict__ counts,
+                       int32_t *__restrict__ offsets, int32_t *__restrict__ rank_offsets,
+                       int32_t *status) {
+    extern __shared__ uint16_t whist[];  // [LT_WARPS][E]
+    __shared__ int s_part[1024];
+    __shared__ int s_tot[1024];
+    __shared__ int s_off[1025];
+    __shared__ int s_wsum[LT_WARPS];
+    __shared__ int s_last;
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int tile = blockIdx.x, T = gridDim.x;
+    for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
+    __syncthreads();
+
+    bool bad = false;
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        int e = -1;
+        if (p < npairs) {
+            e = __ldg(topk_idx + p);
+            if (e < 0 || e >= E) {
+                bad = true;
+                e = -1;
+            }
+        }
+        const unsigned peers = __match_any_sync(FULL, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] += (uint16_t)__popc(peers);
+        __syncwarp();
+    }
+    if (bad) set_status(status, MOE_STATUS_BAD_INDEX);
+    __syncthreads();
+    for (int e = tid; e < E; e += LT_THREADS) {
+        int c = 0;
+#pragma unroll
+        for (int ww = 0; ww < LT_WARPS; ++ww) c += whist[ww * E + e];
+        hist[(size_t)tile * E + e] = c;
+    }
+    // Publish this tile's histogram, then take a ticket; the last ticket scans.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&hdr->ticket, 1u) == (unsigned)(T - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // (A) per-expert sums over groups of tiles; G groups run side by side.
+    int G = LT_THREADS / E;
+    if (G < 1) G = 1;
+    if (G > T) G = T;
+    const int tpg = (T + G - 1) / G;
+    for (int idx = tid; idx < G * E; idx += LT_THREADS) {
+        const int g = idx / E, e = idx - g * E;
+        const int t1 = min(T, (g + 1) * tpg);
+        int c = 0;
+        for (int t = g * tpg; t < t1; ++t) c += __ldcg(hist + (size_t)t * E + e);
+        s_part[idx] = c;
+    }
+    __syncthreads();
+    // (B) exclusive prefix over groups; totals per expert.
+    for (int e = tid; e < E; e += LT_THREADS) {
+        int run = 0;
+        for (int g = 0; g < G; ++g) {
+            const int c = s_part[g * E + e];
+            s_part[g * E + e] = run;
+            run += c;
+        }
+        s_tot[e] = run;
+        counts[e] = run;
+    }
+    __syncthreads();
+    // (C) exclusive prefix over tiles, in place in hist.
+    for (int idx = tid; idx < G * E; idx += LT_THREADS) {
+        const int g = idx / E, e = idx - g * E;
+        const int t1 = min(T, (g + 1) * tpg);
+        int run = s_part[idx];
+        for (int t = g * tpg; t < t1; ++t) {
+            const int c = __ldcg(hist + (size_t)t * E + e);
+            hist[(size_t)t * E + e] = run;
+            run += c;
+        }
+    }
+    // (D) exclusive scan of the padded counts over experts: two experts per thread.
+    const int e0 = 2 * tid, e1 = 2 * tid + 1;
+    const int p0 = e0 < E ? pad_count(s_tot[e0], P) : 0;
+    const int p1 = e1 < E ? pad_count(s_tot[e1], P) : 0;
+    int incl = p0 + p1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = lane < LT_WARPS ? s_wsum[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(FULL, v, off);
+            if (lane >= off) v += o;
+        }
+        if (lane < LT_WARPS) s_wsum[lane] = v;  // inclusive over warps
+    }
+    __syncthreads();
+    const int base = incl - (p0 + p1) + (w > 0 ? s_wsum[w - 1] : 0);
+    if (e0 < E) s_off[e0] = base;
+    if (e1 < E) s_off[e1] = base + p0;
+    if (tid == 0) s_off[E] = s_wsum[LT_WARPS - 1];
+    __syncthreads();
+    for (int e = tid; e <= E; e += LT_THREADS) offsets[e] = s_off[e];
+    const int Eloc = E / R;
+    for (int r = tid; r <= R; r += LT_THREADS) rank_offsets[r] = s_off[r * Eloc];
+    if (tid == 0) {
+        if ((int64_t)s_off[E] > cap) set_status(status, MOE_STATUS_OVERFLOW);
+        hdr->ticket = 0u;  // every other CTA has taken its ticket already
+    }
+}
+
+__global__ void __launch_bounds__(LT_THREADS)
+    layout_slots_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E,
+                        const int32_t *__restrict__ hist, const int32_t *__restrict__ counts,
+                        const int32_t *__restrict__ offsets, int64_t cap,
+                        int32_t *__restrict__ slot_of, int32_t *__restrict__ row_src,
+                        int32_t *status) {
+    extern __shared__ uint16_t whist[];  // [LT_WARPS][E]
+    __shared__ int s_base[1024];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int tile = blockIdx.x;
+    for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
+    __syncthreads();
+
+    int my_e[LT_ITEMS], my_r[LT_ITEMS];
+    const unsigned lt = lanemask_lt();
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        int e = -1;
+        if (p < npairs) {
+            e = __ldg(topk_idx + p);
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned peers = __match_any_sync(FULL, e);
+        const int before = e >= 0 ? (int)whist[w * E + e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
+        __syncwarp();
+        my_e[it] = e;
+        my_r[it] = before + __popc(peers & lt);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += LT_THREADS) {
+        int run = 0;
+#pragma unroll
+        for (int ww = 0; ww < LT_WARPS; ++ww) {
+            const int c = whist[ww * E + e];
+            whist[ww * E + e] = (uint16_t)run;
+            run += c;
+        }
+        s_base[e] = __ldg(offsets + e) + __ldg(hist + (size_t)tile * E + e);
+    }
+    __syncthreads();
+
+    bool over = false;
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        if (p >= npairs) continue;
+        const int e = my_e[it];
+        int s = -1;
+        if (e >= 0) {
+            s = s_base[e] + whist[w * E + e] + my_r[it];
+            if ((int64_t)s >= cap) {
+                s = -1;
+                over = true;
+            }
+        }
+        slot_of[p] = s;
+        if (s >= 0) row_src[s] = p;
+    }
+    if (over) set_status(status, MOE_STATUS_OVERFLOW);
+
+    // Padding rows of each expert, one warp per expert.
+    const int gw = tile * LT_WARPS + w, nw = gridDim.x * LT_WARPS;
+    for (int e = gw; e < E; e += nw) {
+        const int64_t lo = (int64_t)__ldg(offsets + e) + __ldg(counts + e);
+        int64_t hi = __ldg(offsets + e + 1);
+        if (hi > cap) hi = cap;
+        for (int64_t r = lo + lane; r < hi; r += 32) row_src[r] = -1;
+    }
+    // Rows past the layout.
+    const int64_t tail0 = __ldg(offsets + E);
+    for (int64_t r = tail0 + (int64_t)tile * LT_THREADS + tid; r < cap;
+         r += (int64_t)gridDim.x * LT_THREADS)
+        row_src[r] = -1;
+}
+
+cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int P,
+                          int32_t *counts, int32_t *offsets, int32_t *rank_offsets,
+                          int32_t *slot_of, int32_t *row_src, int64_t cap, void *workspace,
+                          int32_t *status, cudaStream_t st) {
+    const int npairs = S * K;
+    const int T = layout_tiles(npairs);
+    auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
+    auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
+    const size_t smem = (size_t)LT_WARPS * E * sizeof(uint16_t);
+    layout_hist_kernel<<<T, LT_THREADS, smem, st>>>(topk_idx, npairs, E, R, P, cap, hist, hdr,
+                                                     counts, offsets, rank_offsets, status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    layout_slots_kernel<<<T, LT_THREADS, smem, st>>>(topk_idx, npairs, E, hist, counts, offsets, cap,
+                                                      slot_of, row_src, status);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

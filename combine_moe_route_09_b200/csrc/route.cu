@@ -1,0 +1,107 @@
+// Router top-K gating: one warp per logits row.
+//
+// "Efficient and portable mixture-of-experts communication", Introduction:
+// each token is sent to the K experts with the highest router scores, and the
+// expert outputs are added with weights from the router's distribution.
+//
+// Each lane holds ceil(E/32) logits of the row in registers as 64-bit keys
+//   key = ordered(logit) << 32 | (0xffffffff - expert)
+// where ordered() maps fp32 to uint32 monotonically (after -0.0 -> +0.0), so a
+// larger key is a larger logit, and on equal logits the lower expert id.  K
+// rounds of a warp-wide max pick the experts in order; the winning key is then
+// cleared.  The softmax over the K selected logits runs on lanes 0..K-1.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ uint32_t ordered_bits(float v) {
+    uint32_t u = __float_as_uint(v);
+    if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_ordered(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+template <int NPER>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int S,
+                                                         int E, int K, int32_t *__restrict__ topk_idx,
+                                                         float *__restrict__ topk_w) {
+    const int lane = threadIdx.x & 31;
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
+        const float *row = logits + (size_t)t * E;
+        unsigned long long key[NPER];
+#pragma unroll
+        for (int j = 0; j < NPER; ++j) {
+            const int e = lane + 32 * j;
+            key[j] = 0ull;  // below every real key
+            if (e < E) {
+                key[j] = ((unsigned long long)ordered_bits(__ldg(row + e)) << 32) |
+                         (unsigned long long)(0xffffffffu - (uint32_t)e);
+            }
+        }
+        float my_logit = 0.f;
+        int my_e = 0;
+        float top = 0.f;
+        for (int k = 0; k < K; ++k) {
+            unsigned long long best = key[0];
+#pragma unroll
+            for (int j = 1; j < NPER; ++j) best = key[j] > best ? key[j] : best;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                unsigned long long o = __shfl_xor_sync(FULL, best, off);
+                best = o > best ? o : best;
+            }
+            const int e = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
+            const float v = from_ordered((uint32_t)(best >> 32));
+            if (k == 0) top = v;
+            if (lane == k) {
+                my_logit = v;
+                my_e = e;
+            }
+            // Keys are unique (they carry the expert id), so exactly one
+            // register in one lane matches the winner; clearing by value keeps
+            // the key array in registers.
+#pragma unroll
+            for (int j = 0; j < NPER; ++j) key[j] = key[j] == best ? 0ull : key[j];
+        }
+        float ex = lane < K ? expf(my_logit - top) : 0.f;
+        float sum = ex;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+        if (lane < K) {
+            topk_idx[(size_t)t * K + lane] = my_e;
+            topk_w[(size_t)t * K + lane] = __fdiv_rn(ex, sum);
+        }
+    }
+}
+
+template <int NPER>
+static cudaError_t launch_route(const float *logits, int S, int E, int K, int32_t *idx, float *w,
+                                cudaStream_t st, int sms) {
+    const int threads = 256;
+    int blocks = (S + 7) / 8;
+    const int cap_blocks = sms * 8;
+    if (blocks > cap_blocks) blocks = cap_blocks;
+    if (blocks < 1) blocks = 1;
+    route_topk_kernel<NPER><<<blocks, threads, 0, st>>>(logits, S, E, K, idx, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t *idx, float *w,
+                              cudaStream_t st, int sms) {
+    const int nper = (E + 31) / 32;
+    if (nper <= 1) return launch_route<1>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 2) return launch_route<2>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 4) return launch_route<4>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 8) return launch_route<8>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 12) return launch_route<12>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 16) return launch_route<16>(logits, S, E, K, idx, w, st, sms);
+    if (nper <= 24) return launch_route<24>(logits, S, E, K, idx, w, st, sms);
+    return launch_route<32>(logits, S, E, K, idx, w, st, sms);
+}
+
+}  // namespace moe

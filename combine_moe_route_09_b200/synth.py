@@ -4,8 +4,11 @@ This module only draws random numbers and fixes shapes; it holds none of the
 routing, layout, quantisation or combine arithmetic.  Tests, the oracle and
 the benchmark all take their inputs from here.
 
-Every tensor gets its own Philox stream (numpy ``SeedSequence(seed).spawn``),
-so a tensor's values do not depend on which other tensors were drawn.  bf16
+Every tensor gets its own stream family (numpy ``SeedSequence(seed).spawn``),
+so a tensor's values do not depend on which other tensors were drawn.  Large
+tensors are drawn in fixed chunks of rows, each chunk from its own SFC64
+stream (spawned from the tensor's seed sequence), in parallel threads; the
+values depend only on (seed, tensor, shape), never on the thread count.  bf16
 tensors are drawn in fp32 and rounded to bf16 (nearest-even) by torch; they
 are returned as numpy ``uint16`` bit patterns.
 
@@ -86,13 +89,42 @@ WORKLOADS = {
                   bias="zipf", seed=5),
 }
 
-# Index of each tensor's Philox stream.
+# Index of each tensor's stream family.
 _STREAMS = dict(logits=0, bias=1, x=2, outliers=3, gains=4, shared=5, residual=6, y=7, perm=8)
 
 
+_CHUNK_ELEMS = 1 << 22
+
+
+def _seq(seed: int, name: str) -> np.random.SeedSequence:
+    return np.random.SeedSequence(seed).spawn(len(_STREAMS))[_STREAMS[name]]
+
+
 def _rng(seed: int, name: str) -> np.random.Generator:
-    ss = np.random.SeedSequence(seed).spawn(len(_STREAMS))[_STREAMS[name]]
-    return np.random.Generator(np.random.Philox(ss))
+    return np.random.Generator(np.random.SFC64(_seq(seed, name)))
+
+
+def _normal(seed: int, name: str, rows: int, cols: int) -> np.ndarray:
+    """N(0,1) fp32 [rows, cols], drawn in fixed row chunks, one SFC64 stream per chunk."""
+    out = np.empty((rows, cols), np.float32)
+    if rows == 0:
+        return out
+    step = max(1, _CHUNK_ELEMS // max(cols, 1))
+    starts = list(range(0, rows, step))
+    seqs = _seq(seed, name).spawn(len(starts))
+
+    def fill(i):
+        r0 = starts[i]
+        g = np.random.Generator(np.random.SFC64(seqs[i]))
+        g.standard_normal(out=out[r0:r0 + step], dtype=np.float32)
+
+    if len(starts) == 1:
+        fill(0)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(len(starts))))
+    return out
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -131,13 +163,13 @@ def expert_bias(w: Workload, alpha: float | None = None) -> np.ndarray:
 
 def logits(w: Workload, alpha: float | None = None) -> np.ndarray:
     """Router logits [S,E] fp32: N(0,1) plus the per-expert bias (added in fp32)."""
-    z = _rng(w.seed, "logits").standard_normal((w.S, w.E), dtype=np.float32)
+    z = _normal(w.seed, "logits", w.S, w.E)
     return (z + expert_bias(w, alpha)[None, :]).astype(np.float32)
 
 
 def activations(w: Workload) -> np.ndarray:
     """Token activations x [S,H] in the workload dtype."""
-    x = _rng(w.seed, "x").standard_normal((w.S, w.H), dtype=np.float32)
+    x = _normal(w.seed, "x", w.S, w.H)
     if w.outlier_frac > 0:
         n = int(round(w.outlier_frac * w.H))
         ch = _rng(w.seed, "outliers").permutation(w.H)[:n]
@@ -146,11 +178,11 @@ def activations(w: Workload) -> np.ndarray:
 
 
 def shared_out(w: Workload) -> np.ndarray:
-    return _cast(_rng(w.seed, "shared").standard_normal((w.S, w.H), dtype=np.float32), w.dtype)
+    return _cast(_normal(w.seed, "shared", w.S, w.H), w.dtype)
 
 
 def residual(w: Workload) -> np.ndarray:
-    return _cast(_rng(w.seed, "residual").standard_normal((w.S, w.H), dtype=np.float32), w.dtype)
+    return _cast(_normal(w.seed, "residual", w.S, w.H), w.dtype)
 
 
 def expert_gains(w: Workload) -> np.ndarray:
@@ -160,7 +192,7 @@ def expert_gains(w: Workload) -> np.ndarray:
 
 def expert_outputs(w: Workload) -> np.ndarray:
     """Expert outputs y [cap,H] ~N(0,1) in the workload dtype (a timing stand-in)."""
-    return _cast(_rng(w.seed, "y").standard_normal((w.cap, w.H), dtype=np.float32), w.dtype)
+    return _cast(_normal(w.seed, "y", w.cap, w.H), w.dtype)
 
 
 def to_torch(a: np.ndarray, dtype: str | None = None, device="cpu"):

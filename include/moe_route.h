@@ -1,0 +1,214 @@
+/*
+ * moe_route.h — C ABI of the B200 (sm_100a) MoE token dispatch / combine library.
+ *
+ * One forward pass of a Mixture-of-Experts layer's routing, on one GPU:
+ *
+ *   moe_route_topk            router top-K gating
+ *   moe_dispatch_layout       per-expert histogram + prefix scan -> padded,
+ *                             expert-contiguous (rank, local expert, slot) layout
+ *   moe_dispatch              scatter token rows into that layout, optionally
+ *                             quantised to FP8 e4m3 with one fp32 scale per
+ *                             128-channel block
+ *   moe_combine_dual_residual gather + top-K weighted sum back to token order,
+ *                             fused with the FarSkip-Collective dual residual
+ *
+ * Sources (page title, section):
+ *   [pplx]    "Efficient and portable mixture-of-experts communication"
+ *             (Perplexity, pplx-kernels): Introduction; Portable Kernels;
+ *             Dispatch; Combine.
+ *   [farskip] Instella-MoE-16B-A3B-SFT / FarSkip-Collective explainer: the dual
+ *             residual stream and its four-line update.
+ *   [deepep]  "DeepSeek AI releases DeepEP": Technical overview (FP8 dispatch).
+ *   [moonep]  "MoonEP developer guide": core API example (Buffer(S, H, K, E,
+ *             num_ep_ranks), dispatch -> tokens_per_expert / cu_seqlens / plan,
+ *             combine(plan, ...)) and tuning parameters (token_padding = 128).
+ *
+ * Notation: S tokens (all R logical ranks together), H hidden size, E experts,
+ * K experts per token, R logical expert-parallel ranks (experts split into R
+ * contiguous blocks of E/R), P = token_padding (0 = none),
+ * cap = rows of the dispatched buffer.  cap = S*K + E*max(P-1, 0) always fits.
+ *
+ * Conventions for every entry point
+ *   - Every pointer except `stream` and those marked "host" is DEVICE memory
+ *     that the caller allocated and owns.  The library allocates nothing,
+ *     keeps no state between calls, and never synchronises with the host:
+ *     all work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns once it is enqueued.
+ *   - Arrays are dense row-major.  Activation buffers (x, xd, y, shared_out,
+ *     residual, outputs) must be 16-byte aligned and their rows a multiple of
+ *     16 bytes (H % 8 == 0 for bf16, H % 4 == 0 for f32, H % 128 == 0 for FP8).
+ *     int32 / fp32 arrays must be 4-byte aligned.
+ *   - Return value: MOE_OK, or MOE_ERR_INVALID_ARG when an argument fails the
+ *     host-side checks stated for the call (nothing is enqueued then), or
+ *     MOE_ERR_CUDA when a launch failed (cudaGetLastError() holds the cause).
+ *   - Problems that only the data reveals (an expert id out of range, a slot
+ *     outside [0, cap), a layout larger than cap) never fault: the offending
+ *     element is skipped and a MOE_STATUS_* bit is OR-ed into *status, a
+ *     device int32 the caller zeroes and reads whenever it likes.  `status`
+ *     may be NULL, in which case such problems are skipped silently.
+ *   - Preconditions that are not checked: finite logits and activations.
+ */
+#ifndef MOE_ROUTE_H
+#define MOE_ROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1
+#define MOE_ERR_CUDA 2
+
+/* element types of activation buffers */
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
+/* dispatch quantisation */
+#define MOE_QUANT_NONE 0
+#define MOE_QUANT_FP8_E4M3_B128 1
+
+/* device status bits (OR-ed into *status) */
+#define MOE_STATUS_BAD_INDEX 1 /* an expert id outside [0, E); that pair was dropped */
+#define MOE_STATUS_OVERFLOW 2  /* the padded layout needs more than cap rows */
+#define MOE_STATUS_BAD_SLOT 4  /* a slot outside [0, cap) reached dispatch/combine; skipped */
+
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 32
+
+/*
+ * Router top-K gating.  [pplx] Introduction: each token goes to the K experts
+ * with the highest router scores; the expert outputs are summed with weights
+ * taken from the router's probability distribution.
+ *
+ *   logits   [S, E] fp32 (device, read)
+ *   topk_idx [S, K] int32 (device, written): the K largest logits of the row
+ *            in descending order; equal logits -> lower expert id first;
+ *            -0.0 and +0.0 are equal.
+ *   topk_w   [S, K] fp32 (device, written): softmax over the K selected
+ *            logits, w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0); this equals
+ *            the full softmax over E renormalised over the chosen K.
+ * Host checks: S >= 0, 1 <= E <= MOE_MAX_EXPERTS, 1 <= K <= min(E, MOE_MAX_TOPK),
+ * non-NULL pointers when S > 0.
+ */
+MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, float *topk_w,
+                   void *stream);
+
+/*
+ * Bytes of scratch memory moe_dispatch_layout needs for these sizes
+ * (a host-side query; no device work).  Returns 0 for invalid sizes.
+ */
+MOE_API size_t moe_dispatch_layout_workspace(int S, int E, int K);
+
+/*
+ * Per-expert histogram and prefix scan into the dispatched layout.
+ * [moonep] core API: dispatch yields tokens_per_expert and cu_seqlens; tuning
+ * parameters: expert groups padded to token_padding rows.  [pplx] Portable
+ * Kernels: a fixed upper bound per (source rank, local expert) receive region
+ * gives every writer a unique address without synchronisation; experts are
+ * split over ranks in blocks of E/R.  [pplx] Dispatch: the receiver records,
+ * per routed token, where it came from, for the combine.
+ *
+ * With pairs i = t*K + k taken in ascending order:
+ *   counts[e]       [E]   int32  number of pairs routed to expert e (tokens_per_expert)
+ *   offsets[e]      [E+1] int32  exclusive scan of the padded counts
+ *                                pc[e] = P ? ceil(counts[e]/P)*P : counts[e] (cu_seqlens)
+ *   rank_offsets[r] [R+1] int32  offsets[r*E/R]: first row of logical rank r
+ *   slot_of[t,k]    [S,K] int32  offsets[e] + number of earlier pairs with the same
+ *                                expert (stable: ascending token, then k); -1 if the
+ *                                pair was dropped (bad index or overflow)
+ *   row_src[s]      [cap] int32  the pair i with slot_of[i] == s, else -1 (padding rows
+ *                                and rows past offsets[E])
+ * The order inside an expert segment is one the pages leave free; ascending
+ * pair order makes the layout deterministic.
+ *
+ * workspace: device scratch of at least moe_dispatch_layout_workspace(S,E,K)
+ *   bytes, 256-byte aligned, owned by the caller.  Its first 256 bytes must be
+ *   zero before the first call; every call leaves them zero again, so one
+ *   zero-filled workspace can serve any number of calls on one stream.  Calls
+ *   that may run concurrently need separate workspaces.
+ * Device status: MOE_STATUS_BAD_INDEX (pair dropped, not counted),
+ *   MOE_STATUS_OVERFLOW (offsets[E] > cap; pairs whose slot would be >= cap
+ *   get slot_of = -1).
+ * Host checks: S >= 0, 1 <= E <= MOE_MAX_EXPERTS, 1 <= K <= MOE_MAX_TOPK, R >= 1,
+ *   E % R == 0, token_padding >= 0, 0 <= cap < 2^31, S*K < 2^31, workspace large
+ *   enough and aligned, non-NULL outputs.
+ */
+MOE_API int moe_dispatch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int token_padding,
+                        int32_t *counts, int32_t *offsets, int32_t *rank_offsets, int32_t *slot_of,
+                        int32_t *row_src, int64_t cap, void *workspace, size_t workspace_bytes,
+                        int32_t *status, void *stream);
+
+/*
+ * Dispatch: scatter each token row into the rows its pairs were given.
+ * [pplx] Dispatch: tokens (with block scaling factors when quantised) are
+ * packed and laid out contiguously per expert for the grouped GEMM.
+ * [deepep] Technical overview: the dispatch may carry FP8.
+ *
+ *   x        [S, H]   dtype (MOE_DTYPE_F32 / MOE_DTYPE_BF16), read
+ *   slot_of  [S, K]   int32, read; negative entries are skipped
+ *   quant == MOE_QUANT_NONE:
+ *     xd     [cap, H] dtype: xd[slot_of[t,k], :] = x[t, :] (bit copy); xs must be NULL
+ *   quant == MOE_QUANT_FP8_E4M3_B128 (H % 128 == 0):
+ *     xd     [cap, H] uint8 e4m3 codes, xs [cap, H/128] fp32 scales.  For block j
+ *            (channels 128j..128j+127) of row t: amax = max |x| (fp32),
+ *            s = amax / 448 (IEEE fp32 division), q = e4m3(x / s) with x / s an
+ *            IEEE fp32 division rounded to nearest even and saturated to +-448;
+ *            s == 0 gives signed zeros.  Every copy of a token carries the same
+ *            bytes and scales.
+ * Rows no pair maps to (padding) are not written.
+ * Device status: MOE_STATUS_BAD_SLOT for a slot >= cap (skipped).
+ * Host checks: S >= 0, H >= 1, 1 <= K <= MOE_MAX_TOPK, dtype/quant known, row
+ * and alignment rules above, xs NULL iff quant == MOE_QUANT_NONE.
+ */
+MOE_API int moe_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
+                 void *xd, float *xs, int64_t cap, int32_t *status, void *stream);
+
+/*
+ * Combine: gather each token's K expert output rows, weight them by the router
+ * weights, and fuse the FarSkip-Collective dual-residual epilogue.
+ * [pplx] Combine: the receiver reads the payloads the routing table names and
+ * takes their router-weighted sum.  [farskip] the dual residual stream:
+ *   residual_no_routed = residual + shared_out
+ *   residual           = residual + mlp_output,  mlp_output = shared_out + routed
+ *
+ *   y          [cap, H] dtype, read (expert outputs in dispatched order)
+ *   slot_of    [S, K] int32, topk_w [S, K] fp32, read
+ *   shared_out [S, H] dtype or NULL;  residual [S, H] dtype or NULL
+ *   residual_out           [S, H] dtype, written
+ *   residual_no_routed_out [S, H] dtype or NULL, written; allowed only when both
+ *                          shared_out and residual are given
+ * Per element, in fp32, in this order:
+ *   acc = 0; for k = 0..K-1 with 0 <= slot < cap: acc = fma(w[t,k], y[slot,h], acc)
+ *   m = shared + acc (or acc);  out = residual + m (or m);  rnr = residual + shared
+ * and each output rounded once to dtype (bf16: nearest even).
+ * residual_out may equal residual (in place); no other buffers may overlap.
+ * Device status: MOE_STATUS_BAD_SLOT for a slot >= cap (skipped).
+ * Host checks: S >= 0, H >= 1, 1 <= K <= MOE_MAX_TOPK, dtype known, row and
+ * alignment rules, residual_no_routed_out only with both shared_out and residual.
+ */
+MOE_API int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int64_t cap,
+                              const int32_t *slot_of, const float *topk_w, const void *shared_out,
+                              const void *residual, void *residual_out,
+                              void *residual_no_routed_out, int32_t *status, void *stream);
+
+/* Human-readable name of a return code (static string, host). */
+MOE_API const char *moe_error_string(int code);
+
+/* Row capacity that always fits the padded layout: S*K + E*max(P-1, 0) (host). */
+MOE_API int64_t moe_capacity(int S, int E, int K, int token_padding);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTE_H */
