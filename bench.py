@@ -294,6 +294,7 @@ def run_ours(args, w, rank, world, local_rank):
     barrier(world)
     torch.cuda.synchronize()
     t_start.record()
+    h0 = time.perf_counter()
     for i in range(K):
         e = ev[i]
         e[0].record()
@@ -306,6 +307,7 @@ def run_ours(args, w, rank, world, local_rank):
         buf.combine(d["y"], sh, rs)
         e[4].record()
     t_end.record()
+    host_us = (time.perf_counter() - h0) / K * 1e6
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
@@ -380,6 +382,7 @@ def run_ours(args, w, rank, world, local_rank):
                              "frac_of_peak": dc_gbs / peak, "frac_of_nominal_8tbs": dc_gbs / 8000.0},
         "phases": phases, "roofline": roofline, "e2e": e2e,
         "gpu_launches": K * buf.KERNELS_PER_STEP, "clocks": clocks,
+        "host_enqueue_us_per_step": host_us,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp)
@@ -396,6 +399,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override S (a smaller case of the same workload, for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -403,6 +408,8 @@ def main(argv=None):
     from combine_moe_route_09_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.replace(S=args.tokens, name=f"{w.name}_S{args.tokens}")
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
         if rank == 0:
