@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe_route.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA = 0, 1, 2
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_QUANT_NONE, MOE_QUANT_FP8_E4M3_B128 = 0, 1
-MOE_STATUS_BAD_INDEX, MOE_STATUS_OVERFLOW, MOE_STATUS_BAD_SLOT = 1, 2, 4
+MOE_STATUS_BAD_INDEX, MOE_STATUS_OVERFLOW, MOE_STATUS_BAD_SLOT, MOE_STATUS_TIMEOUT = 1, 2, 4, 8
 MOE_MAX_EXPERTS, MOE_MAX_TOPK = 1024, 32
 
 _P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t

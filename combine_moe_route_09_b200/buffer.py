@@ -8,9 +8,14 @@ read and write it.  One pass is four calls on one stream, with no host
 synchronisation:
 
     route_topk -> dispatch_layout -> dispatch -> (experts) -> combine_dual_residual
+
+The per-call argument lists for the buffers owned here are built once; an
+input tensor is validated the first time it is seen (and again whenever its
+storage, shape or dtype changes), so a steady-state step costs four C calls.
 """
 from __future__ import annotations
 
+import ctypes
 from typing import Optional
 
 import torch
@@ -26,11 +31,21 @@ class MoeBuffer:
     or bfloat16); fp8 = dispatch quantised to e4m3 with 128-channel scales.
     """
 
+    # kernels one step launches (route 1, layout 2, dispatch 1, combine 1)
+    KERNELS_PER_STEP = 5
+
     def __init__(self, S: int, H: int, K: int, E: int, R: int = 1, token_padding: int = 0,
                  dtype: torch.dtype = torch.bfloat16, fp8: bool = False, device="cuda"):
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError("activations must be float32 or bfloat16")
         self.S, self.H, self.K, self.E, self.R, self.P = S, H, K, E, R, token_padding
-        self.dtype, self.fp8, self.device = dtype, fp8, torch.device(device)
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.dtype, self.fp8, self.device = dtype, fp8, dev
         self.cap = B.moe_capacity(S, E, K, token_padding)
+        if self.cap < 0:
+            raise ValueError("invalid sizes")
         dev = self.device
         i32 = dict(dtype=torch.int32, device=dev)
         self.topk_idx = torch.empty((S, K), **i32)
@@ -49,30 +64,70 @@ class MoeBuffer:
             self.xs = None
         self.out = torch.empty((S, H), dtype=dtype, device=dev)
         self.out_no_routed = torch.empty((S, H), dtype=dtype, device=dev)
+        self._lib = B.lib()
+        self._seen = {}
+        self._dt = B.MOE_DTYPE_F32 if dtype == torch.float32 else B.MOE_DTYPE_BF16
+        p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        L = self.layout
+        self._p_idx, self._p_w, self._p_status = p(self.topk_idx), p(self.topk_w), p(self.status)
+        self._layout_args = (p(self.topk_idx), S, E, K, R, token_padding, p(L.counts), p(L.offsets),
+                             p(L.rank_offsets), p(L.slot_of), p(L.row_src), self.cap,
+                             p(self.workspace), self.workspace.numel(), p(self.status))
+        self._p_slot, self._p_xd = p(L.slot_of), p(self.xd)
+        self._p_xs = p(self.xs) if fp8 else None
+        self._p_out, self._p_rnr = p(self.out), p(self.out_no_routed)
 
     @property
     def quant(self) -> int:
         return B.MOE_QUANT_FP8_E4M3_B128 if self.fp8 else B.MOE_QUANT_NONE
 
+    def _in(self, t: torch.Tensor, name: str, dtypes, shape) -> ctypes.c_void_p:
+        key = (name, t.data_ptr(), tuple(t.shape), t.dtype, t.is_contiguous())
+        ptr = self._seen.get(name)
+        if ptr is None or ptr[0] != key:
+            B._dev(t, name, dtypes, shape)
+            if t.device != self.device:
+                raise ValueError(f"{name} is on {t.device}, buffers are on {self.device}")
+            ptr = (key, ctypes.c_void_p(t.data_ptr()))
+            self._seen[name] = ptr
+        return ptr[1]
+
+    def _stream(self, stream) -> ctypes.c_void_p:
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        return ctypes.c_void_p(s.cuda_stream)
+
     # -- the four calls ---------------------------------------------------------------
     def route(self, logits: torch.Tensor, stream=None):
-        return B.moe_route_topk(logits, self.K, self.topk_idx, self.topk_w, stream=stream)
+        pl = self._in(logits, "logits", (torch.float32,), (self.S, self.E))
+        B._check("moe_route_topk", self._lib.moe_route_topk(pl, self.S, self.E, self.K, self._p_idx,
+                                                             self._p_w, self._stream(stream)))
+        return self.topk_idx, self.topk_w
 
     def plan(self, topk_idx: Optional[torch.Tensor] = None, stream=None) -> B.Layout:
-        idx = self.topk_idx if topk_idx is None else topk_idx
-        return B.moe_dispatch_layout(idx, self.E, self.R, self.P, self.cap, workspace=self.workspace,
-                                     status=self.status, out=self.layout, stream=stream)
+        """Layout of self.topk_idx (or of the given ids, written to this buffer's layout)."""
+        args = self._layout_args
+        if topk_idx is not None:
+            args = (self._in(topk_idx, "topk_idx", (torch.int32,), (self.S, self.K)),) + args[1:]
+        B._check("moe_dispatch_layout", self._lib.moe_dispatch_layout(*args, self._stream(stream)))
+        return self.layout
 
     def dispatch(self, x: torch.Tensor, stream=None):
-        return B.moe_dispatch(x, self.layout.slot_of, self.cap, self.quant, self.xd, self.xs,
-                              status=self.status, stream=stream)
+        px = self._in(x, "x", (self.dtype,), (self.S, self.H))
+        B._check("moe_dispatch", self._lib.moe_dispatch(px, self._dt, self.S, self.H, self.K, self._p_slot,
+                                                         self.quant, self._p_xd, self._p_xs, self.cap,
+                                                         self._p_status, self._stream(stream)))
+        return self.xd, self.xs
 
     def combine(self, y: torch.Tensor, shared_out=None, residual=None, topk_w=None, stream=None):
-        fused = shared_out is not None and residual is not None
-        return B.moe_combine_dual_residual(
-            y, self.layout.slot_of, self.topk_w if topk_w is None else topk_w, shared_out, residual,
-            self.out, self.out_no_routed if fused else None, want_no_routed=fused,
-            status=self.status, stream=stream)
+        py = self._in(y, "y", (self.dtype,), (self.cap, self.H))
+        ps = None if shared_out is None else self._in(shared_out, "shared_out", (self.dtype,), (self.S, self.H))
+        pr = None if residual is None else self._in(residual, "residual", (self.dtype,), (self.S, self.H))
+        pw = self._p_w if topk_w is None else self._in(topk_w, "topk_w", (torch.float32,), (self.S, self.K))
+        fused = ps is not None and pr is not None
+        B._check("moe_combine_dual_residual", self._lib.moe_combine_dual_residual(
+            py, self._dt, self.S, self.H, self.K, self.cap, self._p_slot, pw, ps, pr, self._p_out,
+            self._p_rnr if fused else None, self._p_status, self._stream(stream)))
+        return self.out, (self.out_no_routed if fused else None)
 
     def step(self, logits, x, y, shared_out=None, residual=None, stream=None):
         """One full pass: route, layout, dispatch, combine (y = expert outputs)."""
@@ -80,9 +135,6 @@ class MoeBuffer:
         self.plan(stream=stream)
         self.dispatch(x, stream)
         return self.combine(y, shared_out, residual, stream=stream)
-
-    # kernels one step launches (route 1, layout 2, dispatch 1, combine 1)
-    KERNELS_PER_STEP = 5
 
     def read_status(self) -> int:
         """Reads and clears the device status word (synchronises)."""

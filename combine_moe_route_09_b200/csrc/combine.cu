@@ -7,18 +7,34 @@
 // residual stream:  residual_no_routed = residual + shared_out;
 //                   residual = residual + (shared_out + routed).
 //
-// One warp per token, 16-byte units.  For each unit a lane issues all K
-// gathered loads plus the shared/residual loads before any arithmetic, then
-// accumulates acc = fma(w_k, y_k, acc) in ascending k, adds shared, then
-// residual, and rounds once to the output type.
+// Persistent, warp-specialised kernel.  A work item is one column chunk
+// (`chunk` bytes) of one token; each CTA of a grid sized to the resident CTA
+// count takes a contiguous, balanced share of the items.
+//   producer warp   per token: its K slots and weights (loaded one token
+//                   ahead); per item: the valid mask and weights into the
+//                   stage header, then one TMA bulk copy (cp.async.bulk
+//                   global->shared, completing on the stage's mbarrier) per
+//                   valid slot, plus the shared_out and residual chunks, into
+//                   a ring of STAGES shared-memory stages.  No tensor maps,
+//                   no multicast.
+//   4 consumer warps per item: one 16-byte unit per thread; acc = fma(w_k, y_k,
+//                   acc) in ascending k from shared memory, + shared, +
+//                   residual, round once, 16-byte stores of both streams;
+//                   then release the stage.
+// HBM sees each gathered row chunk, shared_out and residual read once and both
+// outputs written once.  All mbarrier waits are time-bounded.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
-constexpr int CB_THREADS = 256;
-constexpr int CB_WARPS = CB_THREADS / 32;
-constexpr int CB_KCHUNK = 8;  // gathered rows in flight per lane per unit
+constexpr int CB_STAGES = 4;
+constexpr int CB_CONSUMER_WARPS = 4;
+constexpr int CB_CONSUMERS = CB_CONSUMER_WARPS * 32;
+constexpr int CB_THREADS = CB_CONSUMERS + 32;
+constexpr int CB_MAX_CHUNK = CB_CONSUMERS * 16;  // 2048 bytes: one 16-byte unit per consumer
+constexpr int CB_SMEM_BUDGET = 100 * 1024;
 
 template <bool F32>
 struct Vec;
@@ -49,104 +65,200 @@ struct Vec<true> {  // fp32: 4 elements per 16 bytes
     }
 };
 
+struct CombineArgs {
+    const uint8_t *y;
+    const int32_t *slot_of;
+    const float *topk_w;
+    const uint8_t *shared_out;
+    const uint8_t *residual;  // may alias out
+    uint8_t *out;
+    uint8_t *out_no_routed;
+    int32_t *status;
+    int64_t cap;
+    int S, K;
+    int row_bytes;  // H * element size, a multiple of 16
+    int chunk;      // bytes per work item, a multiple of 16, <= CB_MAX_CHUNK
+    int nchunks;    // ceil(row_bytes / chunk)
+};
+
+constexpr int CB_HDR = 256;  // per-stage header: valid mask, then the token's K weights
+
 template <bool F32, bool HAS_SH, bool HAS_RS, bool HAS_RNR>
-__global__ void __launch_bounds__(CB_THREADS)
-    combine_kernel(const uint8_t *__restrict__ y, int S, int nunits, int K, int64_t cap,
-                   const int32_t *__restrict__ slot_of, const float *__restrict__ topk_w,
-                   const uint8_t *__restrict__ shared_out, const uint8_t *residual, uint8_t *out,
-                   uint8_t *__restrict__ out_no_routed, int32_t *status) {
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a) {
     using V = Vec<F32>;
     constexpr int N = V::N;
-    __shared__ int s_slot[CB_WARPS][32];
-    __shared__ float s_w[CB_WARPS][32];
-    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-    const int t = blockIdx.x * CB_WARPS + wl;
-    if (t >= S) return;
-    if (lane < K) {
-        int s = __ldg(slot_of + (size_t)t * K + lane);
-        if ((int64_t)s >= cap) {
-            set_status(status, MOE_STATUS_BAD_SLOT);
-            s = -1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    // [STAGES][header | (K + 2) chunks: K gathered rows, shared_out, residual], then
+    // the full / empty mbarriers of every stage
+    const int K = a.K, chunk = a.chunk;
+    const int stage_bytes = CB_HDR + (K + 2) * chunk;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + CB_STAGES * stage_bytes);
+    const uint32_t smem0 = smem_addr(smem);
+    const uint32_t bar0 = smem_addr(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (CB_STAGES + s); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < CB_STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), CB_CONSUMER_WARPS);
         }
-        s_slot[wl][lane] = s;
-        s_w[wl][lane] = __ldg(topk_w + (size_t)t * K + lane);
+        fence_mbar_init();
     }
-    __syncwarp();
-    const size_t row_bytes = (size_t)nunits * 16;
-    const size_t tok = (size_t)t * row_bytes;
-    for (int u = lane; u < nunits; u += 32) {
-        const size_t ub = (size_t)u * 16;
-        U4 sh, rs;
-        if (HAS_SH) sh = ld_nc_v4(shared_out + tok + ub);
-        if (HAS_RS) rs = *reinterpret_cast<const U4 *>(residual + tok + ub);  // may alias out
-        float acc[N];
-#pragma unroll
-        for (int i = 0; i < N; ++i) acc[i] = 0.f;
-        for (int k0 = 0; k0 < K; k0 += CB_KCHUNK) {
-            U4 v[CB_KCHUNK];
-#pragma unroll
-            for (int kk = 0; kk < CB_KCHUNK; ++kk) {
-                const int k = k0 + kk;
-                const int s = k < K ? s_slot[wl][k] : -1;
-                if (s >= 0) v[kk] = ld_nc_v4(y + (size_t)s * row_bytes + ub);
-            }
-#pragma unroll
-            for (int kk = 0; kk < CB_KCHUNK; ++kk) {
-                const int k = k0 + kk;
-                const int s = k < K ? s_slot[wl][k] : -1;
-                if (s >= 0) {
-                    const float wk = s_w[wl][k];
-                    float f[N];
-                    V::unpack(v[kk], f);
-#pragma unroll
-                    for (int i = 0; i < N; ++i) acc[i] = __fmaf_rn(wk, f[i], acc[i]);
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    // This CTA's items: a contiguous, balanced share, so consecutive items
+    // mostly belong to one token.
+    const long long nitems = (long long)a.S * a.nchunks;
+    const long long first = nitems * blockIdx.x / gridDim.x;
+    const long long last = nitems * (blockIdx.x + 1) / gridDim.x;
+    if (warp == CB_CONSUMER_WARPS) {
+        // ------------------------------- producer -------------------------------
+        // Lane k holds the token's slot k and weight k, loaded one token ahead.
+        int t_cur = -1, cur = -1, nxt = -1;
+        float cur_w = 0.f, nxt_w = 0.f;
+        uint32_t valid = 0;
+        if (first < last && lane < K) {
+            const size_t o = (size_t)(first / a.nchunks) * K + lane;
+            nxt = __ldg(a.slot_of + o);
+            nxt_w = __ldg(a.topk_w + o);
+        }
+        int i = 0;
+        bool ok = true;
+        for (long long item = first; item < last && ok; ++item, ++i) {
+            const int s = i % CB_STAGES;
+            const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+            if (t != t_cur) {
+                t_cur = t;
+                cur = nxt;
+                cur_w = nxt_w;
+                if ((int64_t)cur >= a.cap) {
+                    set_status(a.status, MOE_STATUS_BAD_SLOT);
+                    cur = -1;
+                }
+                valid = __ballot_sync(FULL, cur >= 0);
+                const int tn = t + 1;
+                if (lane < K && (long long)tn * a.nchunks < last) {
+                    nxt = __ldg(a.slot_of + (size_t)tn * K + lane);
+                    nxt_w = __ldg(a.topk_w + (size_t)tn * K + lane);
                 }
             }
+            if (i >= CB_STAGES)
+                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / CB_STAGES) - 1) & 1, a.status));
+            if (!ok) break;
+            const int off = c * chunk;
+            const uint32_t bytes = (uint32_t)min(chunk, a.row_bytes - off);
+            const uint32_t stage = smem0 + (uint32_t)(s * stage_bytes);
+            if (lane < K)
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(stage + 4u + 4u * lane), "f"(cur_w) : "memory");
+            if (lane == 0) asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage), "r"(valid) : "memory");
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t n = (uint32_t)__popc(valid) + (HAS_SH ? 1u : 0u) + (HAS_RS ? 1u : 0u);
+                mbar_arrive_expect_tx(full_bar(s), n * bytes);
+            }
+            __syncwarp();
+            const uint32_t data = stage + CB_HDR;
+            if (cur >= 0)
+                bulk_g2s(data + (uint32_t)(lane * chunk), a.y + (size_t)cur * a.row_bytes + off, bytes, full_bar(s));
+            const size_t tok = (size_t)t * a.row_bytes + off;
+            if (HAS_SH && lane == 0)
+                bulk_g2s(data + (uint32_t)(K * chunk), a.shared_out + tok, bytes, full_bar(s));
+            if (HAS_RS && lane == 1)
+                bulk_g2s(data + (uint32_t)((K + 1) * chunk), a.residual + tok, bytes, full_bar(s));
         }
-        float fsh[N], frs[N], o[N];
-        if (HAS_SH) V::unpack(sh, fsh);
-        if (HAS_RS) V::unpack(rs, frs);
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-            float m = acc[i];
-            if (HAS_SH) m = __fadd_rn(fsh[i], m);
-            o[i] = HAS_RS ? __fadd_rn(frs[i], m) : m;
+        // Never leave copies in flight: wait (bounded) for every stage still loading.
+        if (lane == 0) {
+            for (int j = i - CB_STAGES; j < i; ++j)
+                if (j >= 0) mbar_wait(full_bar(j % CB_STAGES), (j / CB_STAGES) & 1, a.status);
         }
-        st_v4(out + tok + ub, V::pack(o));
-        if (HAS_RNR) {
-            float n[N];
-#pragma unroll
-            for (int i = 0; i < N; ++i) n[i] = __fadd_rn(frs[i], fsh[i]);
-            st_v4(out_no_routed + tok + ub, V::pack(n));
-        }
+        return;
     }
+
+    // ------------------------------- consumers -------------------------------
+    int i = 0;
+    for (long long item = first; item < last; ++item, ++i) {
+        const int s = i % CB_STAGES;
+        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / CB_STAGES) & 1, a.status))) break;
+        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+        const int off = c * chunk;
+        const int bytes = min(chunk, a.row_bytes - off);
+        const uint32_t stage = smem0 + (uint32_t)(s * stage_bytes);
+        const uint32_t data = stage + CB_HDR;
+        uint32_t valid;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(valid) : "r"(stage) : "memory");
+        const int ub = tid * 16;
+        if (ub < bytes) {
+            float acc[N];
+#pragma unroll
+            for (int e = 0; e < N; ++e) acc[e] = 0.f;
+            for (int k = 0; k < K; ++k) {
+                if (!((valid >> k) & 1u)) continue;
+                float wk;
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(wk) : "r"(stage + 4u + 4u * k) : "memory");
+                float f[N];
+                V::unpack(lds128(data + (uint32_t)(k * chunk + ub)), f);
+#pragma unroll
+                for (int e = 0; e < N; ++e) acc[e] = __fmaf_rn(wk, f[e], acc[e]);
+            }
+            float fsh[N] = {}, frs[N] = {}, o[N];
+            if (HAS_SH) V::unpack(lds128(data + (uint32_t)(K * chunk + ub)), fsh);
+            if (HAS_RS) V::unpack(lds128(data + (uint32_t)((K + 1) * chunk + ub)), frs);
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                float m = acc[e];
+                if (HAS_SH) m = __fadd_rn(fsh[e], m);
+                o[e] = HAS_RS ? __fadd_rn(frs[e], m) : m;
+            }
+            const size_t g = (size_t)t * a.row_bytes + off + ub;
+            st_v4(a.out + g, V::pack(o));
+            if (HAS_RNR) {
+                float n[N];
+#pragma unroll
+                for (int e = 0; e < N; ++e) n[e] = __fadd_rn(frs[e], fsh[e]);
+                st_v4(a.out_no_routed + g, V::pack(n));
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+    }
+}
+
+static int combine_chunk(int K, int row_bytes) {
+    int chunk = CB_MAX_CHUNK;
+    while (chunk > 256 && CB_STAGES * (CB_HDR + (K + 2) * chunk) > CB_SMEM_BUDGET) chunk >>= 1;
+    return chunk < row_bytes ? chunk : row_bytes;
+}
+
+static size_t combine_smem(int K, int chunk) {
+    return (size_t)CB_STAGES * (CB_HDR + (K + 2) * chunk) + 2 * CB_STAGES * 8;
 }
 
 template <bool F32, bool SH, bool RS, bool RNR>
-static void launch_cb(const void *y, int S, int nunits, int K, int64_t cap, const int32_t *slot_of,
-                      const float *w, const void *sh, const void *rs, void *out, void *rnr,
-                      int32_t *status, cudaStream_t st) {
-    const int blocks = (S + CB_WARPS - 1) / CB_WARPS;
-    combine_kernel<F32, SH, RS, RNR><<<blocks, CB_THREADS, 0, st>>>(
-        reinterpret_cast<const uint8_t *>(y), S, nunits, K, cap, slot_of, w,
-        reinterpret_cast<const uint8_t *>(sh), reinterpret_cast<const uint8_t *>(rs),
-        reinterpret_cast<uint8_t *>(out), reinterpret_cast<uint8_t *>(rnr), status);
+static cudaError_t launch_cb(const CombineArgs &a, cudaStream_t st) {
+    auto kern = combine_kernel<F32, SH, RS, RNR>;
+    const size_t smem = combine_smem(a.K, a.chunk);
+    static KernelSlots<decltype(kern)> slots;
+    int sms = 0, per_sm = 0;
+    cudaError_t e = slots.prepare(kern, CB_THREADS, smem, &sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    const long long nitems = (long long)a.S * a.nchunks;
+    long long grid = (long long)sms * per_sm;
+    if (grid > nitems) grid = nitems;
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(CB_THREADS), smem, st, a);
 }
 
 template <bool F32>
-static void launch_cb_dt(const void *y, int S, int nunits, int K, int64_t cap,
-                         const int32_t *slot_of, const float *w, const void *sh, const void *rs,
-                         void *out, void *rnr, int32_t *status, cudaStream_t st) {
-    if (sh && rs && rnr)
-        launch_cb<F32, true, true, true>(y, S, nunits, K, cap, slot_of, w, sh, rs, out, rnr, status, st);
-    else if (sh && rs)
-        launch_cb<F32, true, true, false>(y, S, nunits, K, cap, slot_of, w, sh, rs, out, rnr, status, st);
-    else if (sh)
-        launch_cb<F32, true, false, false>(y, S, nunits, K, cap, slot_of, w, sh, rs, out, rnr, status, st);
-    else if (rs)
-        launch_cb<F32, false, true, false>(y, S, nunits, K, cap, slot_of, w, sh, rs, out, rnr, status, st);
-    else
-        launch_cb<F32, false, false, false>(y, S, nunits, K, cap, slot_of, w, sh, rs, out, rnr, status, st);
+static cudaError_t launch_cb_dt(const CombineArgs &a, cudaStream_t st) {
+    const bool sh = a.shared_out, rs = a.residual, rnr = a.out_no_routed;
+    if (sh && rs && rnr) return launch_cb<F32, true, true, true>(a, st);
+    if (sh && rs) return launch_cb<F32, true, true, false>(a, st);
+    if (sh) return launch_cb<F32, true, false, false>(a, st);
+    if (rs) return launch_cb<F32, false, true, false>(a, st);
+    return launch_cb<F32, false, false, false>(a, st);
 }
 
 cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_t cap,
@@ -155,14 +267,22 @@ cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_
                            cudaStream_t st) {
     if (S == 0) return cudaSuccess;
     const bool f32 = dtype == MOE_DTYPE_F32;
-    const int nunits = (int)(((size_t)H * (f32 ? 4 : 2)) / 16);
-    if (f32)
-        launch_cb_dt<true>(y, S, nunits, K, cap, slot_of, topk_w, shared_out, residual, out,
-                           out_no_routed, status, st);
-    else
-        launch_cb_dt<false>(y, S, nunits, K, cap, slot_of, topk_w, shared_out, residual, out,
-                            out_no_routed, status, st);
-    return cudaGetLastError();
+    CombineArgs a;
+    a.y = reinterpret_cast<const uint8_t *>(y);
+    a.slot_of = slot_of;
+    a.topk_w = topk_w;
+    a.shared_out = reinterpret_cast<const uint8_t *>(shared_out);
+    a.residual = reinterpret_cast<const uint8_t *>(residual);
+    a.out = reinterpret_cast<uint8_t *>(out);
+    a.out_no_routed = reinterpret_cast<uint8_t *>(out_no_routed);
+    a.status = status;
+    a.cap = cap;
+    a.S = S;
+    a.K = K;
+    a.row_bytes = H * (f32 ? 4 : 2);
+    a.chunk = combine_chunk(K, a.row_bytes);
+    a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
+    return f32 ? launch_cb_dt<true>(a, st) : launch_cb_dt<false>(a, st);
 }
 
 }  // namespace moe

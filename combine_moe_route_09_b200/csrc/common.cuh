@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe_route.h"
 
 namespace moe {
@@ -53,6 +55,17 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
     return r;
 }
 
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialisation, so it may start while the kernel
+// before it on the stream is still running.  pdl_wait() blocks until that
+// kernel (and so everything before it) has completed and its memory is
+// visible; no kernel touches its inputs or outputs before it.  pdl_trigger()
+// lets the next kernel start launching; kernels call it only after their own
+// pdl_wait(), so work two launches back is always complete when a kernel
+// starts.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(int32_t *status, int bit) {
     if (status) atomicOr(status, bit);
 }
@@ -63,5 +76,67 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
+
+// Launches a kernel with programmatic stream serialisation (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Per-kernel launch facts, computed once per (device, dynamic shared memory
+// size): opts the kernel in to that much dynamic shared memory and records
+// how many CTAs of it fit on one SM.  A handful of sizes per kernel are cached;
+// beyond that the query simply runs again.  Races between host threads only
+// repeat idempotent driver calls.
+template <typename Kern>
+struct KernelSlots {
+    static constexpr int N = 8;
+    int dev[N] = {-1, -1, -1, -1, -1, -1, -1, -1};
+    size_t smem[N] = {};
+    int sms[N] = {}, per_sm[N] = {};
+    int next = 0;
+
+    cudaError_t prepare(Kern kern, int threads, size_t bytes, int *n_sms, int *n_per_sm) {
+        int d = 0;
+        cudaError_t e = cudaGetDevice(&d);
+        if (e != cudaSuccess) return e;
+        for (int i = 0; i < N; ++i) {
+            if (dev[i] == d && smem[i] == bytes) {
+                *n_sms = sms[i];
+                *n_per_sm = per_sm[i];
+                return cudaSuccess;
+            }
+        }
+        if (bytes > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+            if (e != cudaSuccess) return e;
+        }
+        int s = 0, p = 0;
+        e = cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, d);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p, kern, threads, bytes);
+        if (e != cudaSuccess) return e;
+        if (p < 1) p = 1;
+        const int i = next++ % N;
+        sms[i] = s;
+        per_sm[i] = p;
+        smem[i] = bytes;
+        dev[i] = d;
+        *n_sms = s;
+        *n_per_sm = p;
+        return cudaSuccess;
+    }
+};
 
 }  // namespace moe

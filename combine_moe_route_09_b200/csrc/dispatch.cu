@@ -6,72 +6,171 @@
 // expert for the grouped GEMM.  "DeepSeek AI releases DeepEP", Technical
 // overview: the dispatch may carry FP8.
 //
-// One warp per token: the warp reads the row once (16-byte loads, L1 bypassed)
-// and writes it K times (16-byte stores), so HBM sees S*H*b bytes read and
-// S*K*H*b_out written.  For FP8 a lane owns 16 consecutive channels, so the 8
-// lanes of an aligned lane group own one 128-channel block and reduce its amax
-// with three xor-shuffles; scale and quotient are IEEE fp32 divisions, the
-// conversion is cvt.rn.satfinite.e4m3x2.
+// Both kernels are persistent over work items = (token, column chunk), each
+// CTA taking a contiguous, balanced share, and move rows with TMA bulk copies (cp.async.bulk; no tensor maps, no
+// multicast): each row chunk is read from HBM once and written K times.
+//
+//  dispatch_copy_kernel (no quantisation, bf16 or fp32): one warp per CTA,
+//    a contiguous share of the items.  A ring of shared-memory stages; lane 0
+//    bulk-loads item i+STAGES-1 while the K bulk stores of item i go out
+//    straight from its stage (lane k stores copy k; the token's slots are
+//    loaded one token ahead).  A stage is reloaded only after its stores have
+//    finished reading it (cp.async.bulk.wait_group.read).
+//
+//  dispatch_fp8_kernel: each CTA again takes a contiguous share, so
+//    consecutive items mostly belong to one token.  A producer warp
+//    bulk-loads input chunks into a ring of stages and puts the token's slots
+//    (loaded one token ahead) in each stage's header; 4 consumer warps
+//    quantise: each thread owns 16 channels, the 8 threads of a 128-channel
+//    block reduce amax with xor-shuffles, s = amax / 448 (IEEE division) and
+//    q = e4m3(x / s) with the quotient correctly rounded (Markstein's
+//    correction of x * RN(1/s); plain IEEE division for subnormal s) and
+//    cvt.rn.satfinite.e4m3x2.  Each thread stores its 16 codes K times from
+//    registers (a warp writes 512 contiguous bytes per copy); the block's
+//    lead thread stores the scale.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
-constexpr int DP_THREADS = 256;
-constexpr int DP_WARPS = DP_THREADS / 32;
+// ------------------------------------------------------------------------------------------
+// plain copy
+// ------------------------------------------------------------------------------------------
 
-// Loads the token's K slots into the warp's shared-memory row; bad slots -> -1.
-__device__ __forceinline__ void load_slots(int *s_slot, const int32_t *slot_of, int t, int K,
-                                           int64_t cap, int lane, int32_t *status) {
-    if (lane < K) {
-        int s = __ldg(slot_of + (size_t)t * K + lane);
-        if ((int64_t)s >= cap) {
-            set_status(status, MOE_STATUS_BAD_SLOT);
-            s = -1;
-        }
-        s_slot[lane] = s;
+constexpr int DC_STAGES = 6;
+constexpr int DC_CHUNK = 4096;
+
+struct CopyArgs {
+    const uint8_t *x;
+    const int32_t *slot_of;
+    uint8_t *xd;
+    int32_t *status;
+    int64_t cap;
+    int S, K;
+    int row_bytes, chunk, nchunks;
+};
+
+// Items [first, last) of this CTA: a contiguous, balanced share of n items.
+__device__ __forceinline__ void cta_range(long long n, long long &first, long long &last) {
+    first = n * blockIdx.x / gridDim.x;
+    last = n * (blockIdx.x + 1) / gridDim.x;
+}
+
+__global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DC_STAGES * a.chunk);
+    const uint32_t smem0 = smem_addr(smem), bar0 = smem_addr(bars);
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+        for (int s = 0; s < DC_STAGES; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
     }
     __syncwarp();
-}
+    pdl_wait();
+    pdl_trigger();
 
-// Bit copy of rows of `nunits` 16-byte units (bf16 or fp32 without quantisation).
-template <int UNROLL>
-__global__ void __launch_bounds__(DP_THREADS)
-    dispatch_copy_kernel(const uint8_t *__restrict__ x, int S, int nunits, int K,
-                         const int32_t *__restrict__ slot_of, uint8_t *__restrict__ xd, int64_t cap,
-                         int32_t *status) {
-    __shared__ int s_slot[DP_WARPS][32];
-    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-    const int t = blockIdx.x * DP_WARPS + wl;
-    if (t >= S) return;
-    load_slots(s_slot[wl], slot_of, t, K, cap, lane, status);
-    const size_t row_bytes = (size_t)nunits * 16;
-    const uint8_t *src = x + (size_t)t * row_bytes;
-    for (int u0 = 0; u0 < nunits; u0 += 32 * UNROLL) {
-        U4 v[UNROLL];
-#pragma unroll
-        for (int j = 0; j < UNROLL; ++j) {
-            const int u = u0 + 32 * j + lane;
-            if (u < nunits) v[j] = ld_nc_v4(src + (size_t)u * 16);
-        }
-        for (int k = 0; k < K; ++k) {
-            const int s = s_slot[wl][k];
-            if (s < 0) continue;
-            uint8_t *dst = xd + (size_t)s * row_bytes;
-#pragma unroll
-            for (int j = 0; j < UNROLL; ++j) {
-                const int u = u0 + 32 * j + lane;
-                if (u < nunits) st_v4(dst + (size_t)u * 16, v[j]);
+    long long first, last;
+    cta_range((long long)a.S * a.nchunks, first, last);
+    const int n = (int)(last - first);
+    auto load = [&](int j) {  // lane 0 only
+        const long long item = first + j;
+        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+        const int off = c * a.chunk;
+        const uint32_t bytes = (uint32_t)min(a.chunk, a.row_bytes - off);
+        const uint32_t bar = bar0 + 8u * (j % DC_STAGES);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(smem0 + (uint32_t)((j % DC_STAGES) * a.chunk), a.x + (size_t)t * a.row_bytes + off, bytes, bar);
+    };
+    if (lane == 0)
+        for (int j = 0; j < DC_STAGES - 1 && j < n; ++j) load(j);
+    int issued = min(DC_STAGES - 1, n);  // loads issued (lane 0's count, kept uniform)
+
+    // Lane k holds the current token's slot k; the next token's is loaded ahead.
+    int t_cur = -1, cur = -1, nxt = -1;
+    if (n > 0 && lane < a.K) nxt = __ldg(a.slot_of + (size_t)(first / a.nchunks) * a.K + lane);
+    bool ok = true;
+    int i = 0;
+    for (; i < n; ++i) {
+        const long long item = first + i;
+        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+        if (t != t_cur) {
+            t_cur = t;
+            cur = nxt;
+            if ((int64_t)cur >= a.cap) {
+                set_status(a.status, MOE_STATUS_BAD_SLOT);
+                cur = -1;
             }
+            if (lane < a.K && (long long)(t + 1) * a.nchunks < last)
+                nxt = __ldg(a.slot_of + (size_t)(t + 1) * a.K + lane);
+        }
+        const int off = c * a.chunk;
+        const uint32_t bytes = (uint32_t)min(a.chunk, a.row_bytes - off);
+        const int s = i % DC_STAGES;
+        ok = __all_sync(FULL, mbar_wait(bar0 + 8u * s, (i / DC_STAGES) & 1, a.status));
+        if (!ok) break;  // uniform: decided by __all_sync
+        // every lane with a valid slot stores its copy straight from the stage
+        if (cur >= 0) bulk_s2g(a.xd + (size_t)cur * a.row_bytes + off, smem0 + (uint32_t)(s * a.chunk), bytes);
+        bulk_commit();
+        const int j = i + DC_STAGES - 1;
+        if (j < n) {
+            // stage j % STAGES last held item i-1: its stores must have read it
+            bulk_wait_read<1>();
+            __syncwarp();
+            if (lane == 0) load(j);
+            issued = j + 1;
         }
     }
+    // After an early exit, loads i .. issued-1 may still be landing in shared
+    // memory: wait for them (bounded) before the CTA's memory is released.
+    if (!ok && lane == 0)
+        for (int j = i; j < issued; ++j) mbar_wait(bar0 + 8u * (j % DC_STAGES), (j / DC_STAGES) & 1, a.status);
+    bulk_wait_all();
 }
 
-// 16 channels of one lane -> four e4m3x4 words, given the block scale.
+// ------------------------------------------------------------------------------------------
+// FP8 e4m3, 128-channel blocks
+// ------------------------------------------------------------------------------------------
+
+constexpr int DQ_STAGES = 8;
+constexpr int DQ_CONSUMER_WARPS = 4;
+constexpr int DQ_CONSUMERS = DQ_CONSUMER_WARPS * 32;
+constexpr int DQ_THREADS = DQ_CONSUMERS + 32;
+constexpr int DQ_UNIT = 16;                                  // channels per consumer thread
+constexpr int DQ_MAX_BLOCKS = DQ_CONSUMERS * DQ_UNIT / 128;  // 128-channel blocks per item
+constexpr int DQ_HDR = 128;                                  // per-stage header: the token's K slots
+
+struct Fp8Args {
+    const uint8_t *x;
+    const int32_t *slot_of;
+    uint8_t *xd;
+    float *xs;
+    int32_t *status;
+    int64_t cap;
+    int S, H, K;
+    int esz;         // input element bytes (2 or 4)
+    int bpc;         // 128-channel blocks per item (the last item of a row may hold fewer)
+    int nchunks;     // items per token
+    int stage;       // bytes per stage: header + bpc * 128 * esz
+};
+
+// q = x / s rounded to nearest even, for normal x, s: Markstein's correction
+// of x * r with r = 1/s correctly rounded (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990): with r = RN(1/s), q0 = RN(x r) and the remainder
+// e = x - q0 s exact (one fma), RN(q0 + e r) = RN(x / s).  The theorem is
+// about non-zero quotients; for x = -0 the correction yields +0, so the sign
+// of x (the sign of x / s, as s > 0) is copied onto the result.
+__device__ __forceinline__ float div_markstein(float x, float s, float r) {
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, s, x);
+    return copysignf(__fmaf_rn(e, r, q0), x);
+}
+
+// 16 values -> 16 e4m3 codes (value i in byte i), given the block scale s.
 __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
     uint32_t w[4];
     if (s == 0.f) {
-        // amax == 0: every element is a signed zero; keep the sign.
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             uint32_t r = 0;
@@ -79,10 +178,22 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
             for (int b = 0; b < 4; ++b) r |= ((__float_as_uint(f[4 * i + b]) >> 31) << 7) << (8 * b);
             w[i] = r;
         }
-    } else {
+    } else if (s >= 0x1p-90f) {
+        // For |x| >= 2^-102 the remainder x - q0 s is exact, so the quotient is
+        // correctly rounded; smaller x give |x / s| < 2^-11, which is a signed
+        // e4m3 zero whatever its last fp32 bits.  (Checked against IEEE
+        // division over 6e7 inputs: identical codes.)
+        const float r = __frcp_rn(s);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = pack_e4m3x2(__fdiv_rn(f[4 * i + 0], s), __fdiv_rn(f[4 * i + 1], s));
+            const uint32_t lo = pack_e4m3x2(div_markstein(f[4 * i], s, r), div_markstein(f[4 * i + 1], s, r));
+            const uint32_t hi = pack_e4m3x2(div_markstein(f[4 * i + 2], s, r), div_markstein(f[4 * i + 3], s, r));
+            w[i] = lo | (hi << 16);
+        }
+    } else {  // tiny scale: plain IEEE division
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = pack_e4m3x2(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s));
             const uint32_t hi = pack_e4m3x2(__fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
             w[i] = lo | (hi << 16);
         }
@@ -90,105 +201,193 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
     return U4{w[0], w[1], w[2], w[3]};
 }
 
-// FP8 dispatch.  IN_F32: input rows are fp32 (else bf16).  A lane unit is 16
-// channels; nunits = H / 16 is a multiple of 8, so lane groups stay whole.
-template <bool IN_F32, int UNROLL>
-__global__ void __launch_bounds__(DP_THREADS)
-    dispatch_fp8_kernel(const void *__restrict__ x, int S, int H, int K,
-                        const int32_t *__restrict__ slot_of, uint8_t *__restrict__ xd,
-                        float *__restrict__ xs, int64_t cap, int32_t *status) {
-    __shared__ int s_slot[DP_WARPS][32];
-    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-    const int t = blockIdx.x * DP_WARPS + wl;
-    if (t >= S) return;
-    load_slots(s_slot[wl], slot_of, t, K, cap, lane, status);
-    const int nunits = H >> 4, nb = H >> 7;
-    constexpr int LOADS = IN_F32 ? 4 : 2;  // 16-byte loads per unit
-    const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + (size_t)t * H * (IN_F32 ? 4 : 2);
-    for (int u0 = 0; u0 < nunits; u0 += 32 * UNROLL) {
-        U4 raw[UNROLL][LOADS];
-#pragma unroll
-        for (int j = 0; j < UNROLL; ++j) {
-            const int u = u0 + 32 * j + lane;
-            if (u < nunits) {
-#pragma unroll
-                for (int l = 0; l < LOADS; ++l) raw[j][l] = ld_nc_v4(src + (size_t)u * 16 * LOADS + 16 * l);
-            } else {
-#pragma unroll
-                for (int l = 0; l < LOADS; ++l) raw[j][l] = U4{0, 0, 0, 0};
+template <bool IN_F32>
+__global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    // layout: [DQ_STAGES][header (K slots) | bpc*128*esz input bytes] | barriers
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DQ_STAGES * a.stage);
+    const uint32_t smem0 = smem_addr(smem);
+    const uint32_t bar0 = smem_addr(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (DQ_STAGES + s); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < DQ_STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), DQ_CONSUMER_WARPS);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    long long first, last;
+    cta_range((long long)a.S * a.nchunks, first, last);
+    const int row_bytes = a.H * a.esz;
+    const int chunk_bytes = a.bpc * 128 * a.esz;
+    const int nb = a.H >> 7;
+    if (warp == DQ_CONSUMER_WARPS) {
+        // ------------------------------- producer -------------------------------
+        // The token's slots are loaded one token ahead (lane k holds slot k).
+        int t_cur = -1;
+        int nxt = -1;
+        const int t_first = (int)(first / a.nchunks);
+        if (first < last && lane < a.K) nxt = __ldg(a.slot_of + (size_t)t_first * a.K + lane);
+        int cur = -1;
+        int i = 0;
+        bool ok = true;
+        for (long long item = first; item < last && ok; ++item, ++i) {
+            const int s = i % DQ_STAGES;
+            const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+            if (t != t_cur) {
+                t_cur = t;
+                cur = nxt;
+                if ((int64_t)cur >= a.cap) {
+                    set_status(a.status, MOE_STATUS_BAD_SLOT);
+                    cur = -1;
+                }
+                const int tn = t + 1;
+                if (lane < a.K && (long long)tn * a.nchunks < last) nxt = __ldg(a.slot_of + (size_t)tn * a.K + lane);
+            }
+            if (i >= DQ_STAGES)
+                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / DQ_STAGES) - 1) & 1, a.status));
+            if (!ok) break;
+            const int off = c * chunk_bytes;
+            const uint32_t bytes = (uint32_t)min(chunk_bytes, row_bytes - off);
+            const uint32_t st = smem0 + (uint32_t)(s * a.stage);
+            if (lane < a.K) asm volatile("st.shared.s32 [%0], %1;" ::"r"(st + 4u * lane), "r"(cur) : "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(full_bar(s), bytes);
+                bulk_g2s(st + DQ_HDR, a.x + (size_t)t * row_bytes + off, bytes, full_bar(s));
             }
         }
-        U4 q[UNROLL];
-        float scale[UNROLL];
-#pragma unroll
-        for (int j = 0; j < UNROLL; ++j) {
-            float f[16];
+        if (lane == 0) {
+            for (int j = i - DQ_STAGES; j < i; ++j)
+                if (j >= 0) mbar_wait(full_bar(j % DQ_STAGES), (j / DQ_STAGES) & 1, a.status);
+        }
+        return;
+    }
+
+    // ------------------------------- consumers -------------------------------
+    // Thread tid owns channels [16 tid, 16 tid + 16) of the item; the 8 threads
+    // of a 128-channel block reduce its amax.  Codes: one 16-byte store per copy.
+    int i = 0;
+    for (long long item = first; item < last; ++item, ++i) {
+        const int s = i % DQ_STAGES;
+        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / DQ_STAGES) & 1, a.status))) break;
+        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+        const int col0 = c * a.bpc * 128;                   // first channel of the item
+        const int nch = min(a.bpc * 128, a.H - col0);       // channels in this item
+        const bool active = tid * DQ_UNIT < nch;            // whole blocks: groups all-or-nothing
+        const uint32_t st = smem0 + (uint32_t)(s * a.stage);
+        float f[16];
+        if (active) {
+            const uint32_t src = st + DQ_HDR + (uint32_t)(tid * DQ_UNIT * a.esz);
             if (IN_F32) {
 #pragma unroll
                 for (int l = 0; l < 4; ++l) {
-                    f[4 * l + 0] = __uint_as_float(raw[j][l].x);
-                    f[4 * l + 1] = __uint_as_float(raw[j][l].y);
-                    f[4 * l + 2] = __uint_as_float(raw[j][l].z);
-                    f[4 * l + 3] = __uint_as_float(raw[j][l].w);
+                    const U4 v = lds128(src + 16u * l);
+                    f[4 * l + 0] = __uint_as_float(v.x);
+                    f[4 * l + 1] = __uint_as_float(v.y);
+                    f[4 * l + 2] = __uint_as_float(v.z);
+                    f[4 * l + 3] = __uint_as_float(v.w);
                 }
             } else {
 #pragma unroll
                 for (int l = 0; l < 2; ++l) {
-                    f[8 * l + 0] = bf16lo(raw[j][l].x);
-                    f[8 * l + 1] = bf16hi(raw[j][l].x);
-                    f[8 * l + 2] = bf16lo(raw[j][l].y);
-                    f[8 * l + 3] = bf16hi(raw[j][l].y);
-                    f[8 * l + 4] = bf16lo(raw[j][l].z);
-                    f[8 * l + 5] = bf16hi(raw[j][l].z);
-                    f[8 * l + 6] = bf16lo(raw[j][l].w);
-                    f[8 * l + 7] = bf16hi(raw[j][l].w);
+                    const U4 v = lds128(src + 16u * l);
+                    f[8 * l + 0] = bf16lo(v.x); f[8 * l + 1] = bf16hi(v.x);
+                    f[8 * l + 2] = bf16lo(v.y); f[8 * l + 3] = bf16hi(v.y);
+                    f[8 * l + 4] = bf16lo(v.z); f[8 * l + 5] = bf16hi(v.z);
+                    f[8 * l + 6] = bf16lo(v.w); f[8 * l + 7] = bf16hi(v.w);
                 }
             }
-            float amax = 0.f;
+        } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 4));
-            const float s = __fdiv_rn(amax, 448.0f);
-            scale[j] = s;
-            q[j] = quant16(f, s);
+            for (int e = 0; e < 16; ++e) f[e] = 0.f;
         }
-        for (int k = 0; k < K; ++k) {
-            const int s = s_slot[wl][k];
-            if (s < 0) continue;
-            uint8_t *dst = xd + (size_t)s * H;
-            float *sdst = xs + (size_t)s * nb;
+        int myslot = -1;
+        if (lane < a.K) asm volatile("ld.shared.s32 %0, [%1];" : "=r"(myslot) : "r"(st + 4u * lane) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));  // input stage no longer needed
+
+        float amax = 0.f;
 #pragma unroll
-            for (int j = 0; j < UNROLL; ++j) {
-                const int u = u0 + 32 * j + lane;
-                if (u < nunits) {
-                    st_v4(dst + (size_t)u * 16, q[j]);
-                    if ((lane & 7) == 0) sdst[u >> 3] = scale[j];
-                }
-            }
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 4));
+        const float scale = __fdiv_rn(amax, 448.0f);
+        const U4 q = quant16(f, scale);
+
+        const int col = col0 + tid * DQ_UNIT;
+        const bool lead = active && (tid & 7) == 0;
+        const int blk = col >> 7;
+        for (int k = 0; k < a.K; ++k) {
+            const int sl = __shfl_sync(FULL, myslot, k);
+            if (sl < 0) continue;
+            if (active) st_v4(a.xd + (size_t)sl * a.H + col, q);
+            if (lead) a.xs[(size_t)sl * nb + blk] = scale;
         }
     }
+}
+
+// ------------------------------------------------------------------------------------------
+
+template <typename Kern>
+static cudaError_t persistent_grid(KernelSlots<Kern> &slots, Kern kern, int threads, size_t smem,
+                                   long long nitems, unsigned *grid) {
+    int sms = 0, per_sm = 0;
+    cudaError_t e = slots.prepare(kern, threads, smem, &sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    long long g = (long long)sms * per_sm;
+    if (g > nitems) g = nitems;
+    *grid = (unsigned)(g < 1 ? 1 : g);
+    return cudaSuccess;
 }
 
 cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of,
                             int quant, void *xd, float *xs, int64_t cap, int32_t *status,
                             cudaStream_t st) {
     if (S == 0) return cudaSuccess;
-    const int blocks = (S + DP_WARPS - 1) / DP_WARPS;
+    const int esz = dtype == MOE_DTYPE_F32 ? 4 : 2;
+    const int row_bytes = H * esz;
     if (quant == MOE_QUANT_NONE) {
-        const int nunits = (int)(((size_t)H * (dtype == MOE_DTYPE_F32 ? 4 : 2)) / 16);
-        dispatch_copy_kernel<2><<<blocks, DP_THREADS, 0, st>>>(
-            reinterpret_cast<const uint8_t *>(x), S, nunits, K, slot_of,
-            reinterpret_cast<uint8_t *>(xd), cap, status);
-    } else if (dtype == MOE_DTYPE_BF16) {
-        dispatch_fp8_kernel<false, 2><<<blocks, DP_THREADS, 0, st>>>(
-            x, S, H, K, slot_of, reinterpret_cast<uint8_t *>(xd), xs, cap, status);
-    } else {
-        dispatch_fp8_kernel<true, 1><<<blocks, DP_THREADS, 0, st>>>(
-            x, S, H, K, slot_of, reinterpret_cast<uint8_t *>(xd), xs, cap, status);
+        CopyArgs a{reinterpret_cast<const uint8_t *>(x), slot_of, reinterpret_cast<uint8_t *>(xd), status,
+                   cap, S, K, row_bytes, 0, 0};
+        a.chunk = row_bytes < DC_CHUNK ? row_bytes : DC_CHUNK;
+        a.nchunks = (row_bytes + a.chunk - 1) / a.chunk;
+        const size_t smem = (size_t)DC_STAGES * a.chunk + DC_STAGES * 8;
+        static KernelSlots<decltype(&dispatch_copy_kernel)> slots;
+        unsigned grid = 1;
+        cudaError_t e = persistent_grid(slots, &dispatch_copy_kernel, 32, smem, (long long)S * a.nchunks, &grid);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(dispatch_copy_kernel, dim3(grid), dim3(32), smem, st, a);
     }
-    return cudaGetLastError();
+    Fp8Args a{reinterpret_cast<const uint8_t *>(x), slot_of, reinterpret_cast<uint8_t *>(xd), xs, status,
+              cap, S, H, K, esz, 0, 0, 0};
+    // Split each row into the fewest items of at most DQ_MAX_BLOCKS blocks, as evenly as possible.
+    const int blocks = H / 128;
+    const int n = (blocks + DQ_MAX_BLOCKS - 1) / DQ_MAX_BLOCKS;
+    a.bpc = (blocks + n - 1) / n;
+    a.nchunks = (blocks + a.bpc - 1) / a.bpc;
+    a.stage = DQ_HDR + a.bpc * 128 * esz;
+    const size_t smem = (size_t)DQ_STAGES * a.stage + 2 * DQ_STAGES * 8;
+    unsigned grid = 1;
+    cudaError_t e;
+    if (dtype == MOE_DTYPE_BF16) {
+        static KernelSlots<decltype(&dispatch_fp8_kernel<false>)> slots;
+        e = persistent_grid(slots, &dispatch_fp8_kernel<false>, DQ_THREADS, smem, (long long)S * a.nchunks, &grid);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(dispatch_fp8_kernel<false>, dim3(grid), dim3(DQ_THREADS), smem, st, a);
+    }
+    static KernelSlots<decltype(&dispatch_fp8_kernel<true>)> slots;
+    e = persistent_grid(slots, &dispatch_fp8_kernel<true>, DQ_THREADS, smem, (long long)S * a.nchunks, &grid);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(dispatch_fp8_kernel<true>, dim3(grid), dim3(DQ_THREADS), smem, st, a);
 }
 
 }  // namespace moe

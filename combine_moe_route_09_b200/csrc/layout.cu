@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(LT_THREADS)
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int tile = blockIdx.x, T = gridDim.x;
     for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
+    pdl_wait();
+    pdl_trigger();
     __syncthreads();
 
     bool bad = false;
@@ -170,6 +172,11 @@ __global__ void __launch_bounds__(LT_THREADS)
     for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
     __syncthreads();
 
+    // Before pdl_wait: this kernel follows layout_hist in the same call, and
+    // layout_hist triggered only after its own wait, so topk_idx (written two
+    // launches back or earlier) is complete; layout_hist only reads it.  The
+    // rank computation below therefore overlaps layout_hist's scan.  Loads go
+    // through L2 (ld.global.cg), never a stale L1 line.
     int my_e[LT_ITEMS], my_r[LT_ITEMS];
     const unsigned lt = lanemask_lt();
 #pragma unroll
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(LT_THREADS)
         const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
         int e = -1;
         if (p < npairs) {
-            e = __ldg(topk_idx + p);
+            e = __ldcg(topk_idx + p);
             if (e < 0 || e >= E) e = -1;
         }
         const unsigned peers = __match_any_sync(FULL, e);
@@ -197,8 +204,11 @@ __global__ void __launch_bounds__(LT_THREADS)
             whist[ww * E + e] = (uint16_t)run;
             run += c;
         }
-        s_base[e] = __ldg(offsets + e) + __ldg(hist + (size_t)tile * E + e);
     }
+    pdl_wait();  // offsets, counts and the tile prefixes come from layout_hist
+    pdl_trigger();
+    for (int e = tid; e < E; e += LT_THREADS)
+        s_base[e] = __ldcg(offsets + e) + __ldcg(hist + (size_t)tile * E + e);
     __syncthreads();
 
     bool over = false;
@@ -223,13 +233,13 @@ __global__ void __launch_bounds__(LT_THREADS)
     // Padding rows of each expert, one warp per expert.
     const int gw = tile * LT_WARPS + w, nw = gridDim.x * LT_WARPS;
     for (int e = gw; e < E; e += nw) {
-        const int64_t lo = (int64_t)__ldg(offsets + e) + __ldg(counts + e);
-        int64_t hi = __ldg(offsets + e + 1);
+        const int64_t lo = (int64_t)__ldcg(offsets + e) + __ldcg(counts + e);
+        int64_t hi = __ldcg(offsets + e + 1);
         if (hi > cap) hi = cap;
         for (int64_t r = lo + lane; r < hi; r += 32) row_src[r] = -1;
     }
     // Rows past the layout.
-    const int64_t tail0 = __ldg(offsets + E);
+    const int64_t tail0 = __ldcg(offsets + E);
     for (int64_t r = tail0 + (int64_t)tile * LT_THREADS + tid; r < cap;
          r += (int64_t)gridDim.x * LT_THREADS)
         row_src[r] = -1;
@@ -244,13 +254,12 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
     const size_t smem = (size_t)LT_WARPS * E * sizeof(uint16_t);
-    layout_hist_kernel<<<T, LT_THREADS, smem, st>>>(topk_idx, npairs, E, R, P, cap, hist, hdr,
-                                                     counts, offsets, rank_offsets, status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(layout_hist_kernel, dim3(T), dim3(LT_THREADS), smem, st, topk_idx, npairs,
+                                 E, R, P, cap, hist, hdr, counts, offsets, rank_offsets, status);
     if (err != cudaSuccess) return err;
-    layout_slots_kernel<<<T, LT_THREADS, smem, st>>>(topk_idx, npairs, E, hist, counts, offsets, cap,
-                                                      slot_of, row_src, status);
-    return cudaGetLastError();
+    return launch_pdl(layout_slots_kernel, dim3(T), dim3(LT_THREADS), smem, st, topk_idx, npairs, E,
+                      (const int32_t *)hist, (const int32_t *)counts, (const int32_t *)offsets, cap, slot_of,
+                      row_src, status);
 }
 
 }  // namespace moe

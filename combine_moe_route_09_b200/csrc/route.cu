@@ -4,12 +4,14 @@
 // each token is sent to the K experts with the highest router scores, and the
 // expert outputs are added with weights from the router's distribution.
 //
-// Each lane holds ceil(E/32) logits of the row in registers as 64-bit keys
-//   key = ordered(logit) << 32 | (0xffffffff - expert)
-// where ordered() maps fp32 to uint32 monotonically (after -0.0 -> +0.0), so a
-// larger key is a larger logit, and on equal logits the lower expert id.  K
-// rounds of a warp-wide max pick the experts in order; the winning key is then
-// cleared.  The softmax over the K selected logits runs on lanes 0..K-1.
+// Each lane holds ceil(E/32) logits of the row (expert e = lane + 32*j) in
+// registers as ordered 32-bit keys: ordered() maps fp32 to uint32
+// monotonically (after -0.0 -> +0.0), so a larger key is a larger logit.
+// Round k of K: the warp max of the keys (redux.sync.max), then the lowest
+// expert id holding that key (redux.sync.min over each lane's lowest
+// candidate) -- ties go to the lower id -- and that key is cleared to 0,
+// below every real key.  The softmax over the K selected logits runs on lanes
+// 0..K-1.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -29,46 +31,38 @@ template <int NPER>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int S,
                                                          int E, int K, int32_t *__restrict__ topk_idx,
                                                          float *__restrict__ topk_w) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
         const float *row = logits + (size_t)t * E;
-        unsigned long long key[NPER];
+        uint32_t key[NPER];
 #pragma unroll
         for (int j = 0; j < NPER; ++j) {
             const int e = lane + 32 * j;
-            key[j] = 0ull;  // below every real key
-            if (e < E) {
-                key[j] = ((unsigned long long)ordered_bits(__ldg(row + e)) << 32) |
-                         (unsigned long long)(0xffffffffu - (uint32_t)e);
-            }
+            key[j] = e < E ? ordered_bits(__ldg(row + e)) : 0u;
         }
-        float my_logit = 0.f;
+        uint32_t my_key = 0, top = 0;
         int my_e = 0;
-        float top = 0.f;
         for (int k = 0; k < K; ++k) {
-            unsigned long long best = key[0];
+            uint32_t m = key[0];
 #pragma unroll
-            for (int j = 1; j < NPER; ++j) best = key[j] > best ? key[j] : best;
+            for (int j = 1; j < NPER; ++j) m = max(m, key[j]);
+            const uint32_t best = __reduce_max_sync(FULL, m);
+            uint32_t cand = 0xffffffffu;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                unsigned long long o = __shfl_xor_sync(FULL, best, off);
-                best = o > best ? o : best;
-            }
-            const int e = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
-            const float v = from_ordered((uint32_t)(best >> 32));
-            if (k == 0) top = v;
+            for (int j = NPER - 1; j >= 0; --j) cand = key[j] == best ? (uint32_t)(lane + 32 * j) : cand;
+            const uint32_t win = __reduce_min_sync(FULL, cand);
+            if (k == 0) top = best;
             if (lane == k) {
-                my_logit = v;
-                my_e = e;
+                my_key = best;
+                my_e = (int)win;
             }
-            // Keys are unique (they carry the expert id), so exactly one
-            // register in one lane matches the winner; clearing by value keeps
-            // the key array in registers.
 #pragma unroll
-            for (int j = 0; j < NPER; ++j) key[j] = key[j] == best ? 0ull : key[j];
+            for (int j = 0; j < NPER; ++j) key[j] = (uint32_t)(lane + 32 * j) == win ? 0u : key[j];
         }
-        float ex = lane < K ? expf(my_logit - top) : 0.f;
+        const float ex = lane < K ? expf(from_ordered(my_key) - from_ordered(top)) : 0.f;
         float sum = ex;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
@@ -87,8 +81,7 @@ static cudaError_t launch_route(const float *logits, int S, int E, int K, int32_
     const int cap_blocks = sms * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
     if (blocks < 1) blocks = 1;
-    route_topk_kernel<NPER><<<blocks, threads, 0, st>>>(logits, S, E, K, idx, w);
-    return cudaGetLastError();
+    return launch_pdl(route_topk_kernel<NPER>, dim3(blocks), dim3(threads), 0, st, logits, S, E, K, idx, w);
 }
 
 cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t *idx, float *w,

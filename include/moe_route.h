@@ -46,6 +46,9 @@
  *     element is skipped and a MOE_STATUS_* bit is OR-ed into *status, a
  *     device int32 the caller zeroes and reads whenever it likes.  `status`
  *     may be NULL, in which case such problems are skipped silently.
+ *   - Every wait inside a kernel (pipeline barriers between the copy engine
+ *     and the compute threads) is bounded in time; one that expires sets
+ *     MOE_STATUS_TIMEOUT and the kernel returns instead of hanging.
  *   - Preconditions that are not checked: finite logits and activations.
  */
 #ifndef MOE_ROUTE_H
@@ -81,6 +84,7 @@ extern "C" {
 #define MOE_STATUS_BAD_INDEX 1 /* an expert id outside [0, E); that pair was dropped */
 #define MOE_STATUS_OVERFLOW 2  /* the padded layout needs more than cap rows */
 #define MOE_STATUS_BAD_SLOT 4  /* a slot outside [0, cap) reached dispatch/combine; skipped */
+#define MOE_STATUS_TIMEOUT 8   /* an internal pipeline wait exceeded its time bound; output incomplete */
 
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_TOPK 32

@@ -246,3 +246,36 @@ def test_invalid_args_raise_before_launch():
     lg = torch.zeros((8, 4), dtype=torch.float32, device="cuda")
     with pytest.raises(B.MoeError):
         B.moe_route_topk(lg, 5)
+
+
+def _midpoint_blocks(rng, S, H, in_bf16: bool):
+    """Rows whose quotients x/s sit within a few fp32 ulps of e4m3 rounding midpoints."""
+    codes = np.arange(0, 0x7E, dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    mids = (vals[:-1] + vals[1:]) / 2
+    x = np.empty((S, H), np.float32)
+    for t in range(S):
+        for b in range(H // 128):
+            a = np.float32(rng.uniform(0.5, 4.0) * 2.0 ** int(rng.integers(-20, 21)))
+            if in_bf16:
+                a = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.array([a], np.float32)))[0]
+            s = np.float32(a) / np.float32(448.0)
+            m = rng.choice(mids, 127) * rng.choice([-1.0, 1.0], 127)
+            v = (m * np.float64(s)).astype(np.float32)
+            v = (v.view(np.int32) + rng.integers(-2, 3, 127).astype(np.int32)).view(np.float32)
+            blk = np.concatenate([[a], v]).astype(np.float32)
+            rng.shuffle(blk)
+            x[t, 128 * b:128 * (b + 1)] = blk
+    return synth.f32_to_bf16_bits(x) if in_bf16 else x
+
+
+@pytest.mark.parametrize("in_bf16", [False, True])
+def test_fp8_quotients_near_rounding_midpoints(in_bf16):
+    rng = np.random.default_rng(8 + in_bf16)
+    S, H, K = 96, 1024, 3
+    x = _midpoint_blocks(rng, S, H, in_bf16)
+    slot = np.arange(S * K, dtype=np.int32).reshape(S, K)
+    ref_xd, ref_xs = oracle.dispatch(x, slot, S * K, quant=oracle.QUANT_FP8_E4M3_B128)
+    gxd, gxs = B.moe_dispatch(dev(x), dev(slot), S * K, B.MOE_QUANT_FP8_E4M3_B128)
+    np.testing.assert_array_equal(host(gxs), ref_xs)
+    np.testing.assert_array_equal(host(gxd), ref_xd)
