@@ -17,7 +17,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_route.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA = 0, 1, 2
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA, MOE_ERR_SCRATCH_TOO_SMALL = 0, 1, 2, 3
+MOE_STATIC_LAYOUT_SCRATCH_BYTES = 1 << 20
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_QUANT_NONE, MOE_QUANT_FP8_E4M3_B128 = 0, 1
 MOE_STATUS_BAD_INDEX, MOE_STATUS_OVERFLOW, MOE_STATUS_BAD_SLOT, MOE_STATUS_TIMEOUT = 1, 2, 4, 8
@@ -32,6 +33,7 @@ SIGNATURES = {
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _Z, _P, _P]),
     "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
     "moe_combine_dual_residual": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch_layout_static": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _P]),
     "moe_error_string": (ctypes.c_char_p, [_I]),
     "moe_capacity": (_L, [_I, _I, _I, _I]),
 }
@@ -154,6 +156,33 @@ def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, token_padding: i
         _ptr(topk_idx), S, E, K, R, token_padding, _ptr(out.counts), _ptr(out.offsets),
         _ptr(out.rank_offsets), _ptr(out.slot_of), _ptr(out.row_src), cap, _ptr(workspace),
         workspace.numel(), _ptr(status), _stream(stream, dev)))
+    return out._replace(cap=cap)
+
+
+def moe_dispatch_layout_static(topk_idx: torch.Tensor, E: int, R: int, token_padding: int = 0,
+                               cap: Optional[int] = None, *, status=None, out=None,
+                               stream=None) -> Layout:
+    """moe_dispatch_layout without a workspace, for callers that may not allocate
+    device memory where they call it: the scratch is an array built into the
+    library (MOE_STATIC_LAYOUT_SCRATCH_BYTES per GPU).  Outputs are allocated here
+    only when ``out`` is not given.  Calls that may overlap on the GPU share that
+    array and must be serialised; the first call on a device should precede any
+    stream capture."""
+    _dev(topk_idx, "topk_idx", (torch.int32,))
+    S, K = topk_idx.shape
+    dev = topk_idx.device
+    if cap is None:
+        cap = moe_capacity(S, E, K, token_padding)
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                     torch.empty((S, K), **i32), torch.empty(max(cap, 0), **i32), cap)
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_dispatch_layout_static", lib().moe_dispatch_layout_static(
+        _ptr(topk_idx), S, E, K, R, token_padding, _ptr(out.counts), _ptr(out.offsets),
+        _ptr(out.rank_offsets), _ptr(out.slot_of), _ptr(out.row_src), cap, _ptr(status),
+        _stream(stream, dev)))
     return out._replace(cap=cap)
 
 

@@ -34,6 +34,8 @@ const char *moe_error_string(int code) {
         case MOE_OK: return "ok";
         case MOE_ERR_INVALID_ARG: return "invalid argument";
         case MOE_ERR_CUDA: return "CUDA launch error";
+        case MOE_ERR_SCRATCH_TOO_SMALL:
+            return "sizes need more scratch than moe_dispatch_layout_static's built-in array";
         default: return "unknown error";
     }
 }

@@ -71,6 +71,7 @@ extern "C" {
 #define MOE_OK 0
 #define MOE_ERR_INVALID_ARG 1
 #define MOE_ERR_CUDA 2
+#define MOE_ERR_SCRATCH_TOO_SMALL 3 /* sizes need more scratch than moe_dispatch_layout_static has */
 
 /* element types of activation buffers */
 #define MOE_DTYPE_F32 0
@@ -204,6 +205,36 @@ MOE_API int moe_combine_dual_residual(const void *y, int dtype, int S, int H, in
                               const int32_t *slot_of, const float *topk_w, const void *shared_out,
                               const void *residual, void *residual_out,
                               void *residual_no_routed_out, int32_t *status, void *stream);
+
+/*
+ * moe_dispatch_layout_static: the same layout as moe_dispatch_layout, for a
+ * caller that cannot allocate device memory where it makes this call -- e.g. a
+ * host framework or engine plugin that owns all device memory up front and
+ * forbids allocation while it executes, or a latency-critical loop that must
+ * not pay for cudaMalloc, which may synchronise the device.  (The pages have
+ * no counterpart; this is a convenience of this library.)
+ *
+ * Arguments, outputs, device status and host checks are those of
+ * moe_dispatch_layout without `workspace` / `workspace_bytes`.  The scratch is
+ * a MOE_STATIC_LAYOUT_SCRATCH_BYTES array inside the library, held by every
+ * GPU that loads the library until the process exits; sizes with
+ * moe_dispatch_layout_workspace(S, E, K) > MOE_STATIC_LAYOUT_SCRATCH_BYTES
+ * are refused with MOE_ERR_SCRATCH_TOO_SMALL (the limit is about 2 million
+ * (token, k) pairs at E = 256, 8 million at E = 64).  Nothing is allocated: no
+ * cudaMalloc, no cudaFree.
+ *
+ * The first call on a device looks up the array's device address there
+ * (cudaGetSymbolAddress, with that device current), so make that first call
+ * before any stream capture.  Every call on a device shares the one array and
+ * clears its zero-initialised part on `stream` first; calls whose work may
+ * overlap on the GPU (other streams, other host threads) race on it and must
+ * be serialised by the caller.
+ */
+#define MOE_STATIC_LAYOUT_SCRATCH_BYTES (1 << 20)
+MOE_API int moe_dispatch_layout_static(const int32_t *topk_idx, int S, int E, int K, int R,
+                                       int token_padding, int32_t *counts, int32_t *offsets,
+                                       int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src,
+                                       int64_t cap, int32_t *status, void *stream);
 
 /* Human-readable name of a return code (static string, host). */
 MOE_API const char *moe_error_string(int code);
