@@ -128,9 +128,9 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
         }
         int i = 0;
         bool ok = true;
-        for (long long item = first; item < last && ok; ++item, ++i) {
+        int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
+        for (long long item = first; item < last && ok; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
             const int s = i % CB_STAGES;
-            const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
             if (t != t_cur) {
                 t_cur = t;
                 cur = nxt;
@@ -180,10 +180,10 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
 
     // ------------------------------- consumers -------------------------------
     int i = 0;
-    for (long long item = first; item < last; ++item, ++i) {
+    int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
+    for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
         const int s = i % CB_STAGES;
         if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / CB_STAGES) & 1, a.status))) break;
-        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
         const int off = c * chunk;
         const int bytes = min(chunk, a.row_bytes - off);
         const uint32_t stage = smem0 + (uint32_t)(s * stage_bytes);

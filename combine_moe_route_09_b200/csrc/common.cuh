@@ -122,6 +122,12 @@ struct KernelSlots {
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
             if (e != cudaSuccess) return e;
         }
+        // Every kernel of the library asks for the largest shared-memory
+        // carveout, so consecutive kernels never wait for an L1/shared split
+        // to be reconfigured.
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         int s = 0, p = 0;
         e = cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, d);
         if (e != cudaSuccess) return e;

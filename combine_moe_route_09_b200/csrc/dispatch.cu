@@ -73,17 +73,26 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
     long long first, last;
     cta_range((long long)a.S * a.nchunks, first, last);
     const int n = (int)(last - first);
-    auto load = [&](int j) {  // lane 0 only
-        const long long item = first + j;
-        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
-        const int off = c * a.chunk;
+    // Loads run DC_STAGES - 1 items ahead of the stores; each side walks its
+    // (token, chunk) pair incrementally.
+    int lt = (int)(first / a.nchunks), lc = (int)(first - (long long)lt * a.nchunks);
+    auto load = [&](int j) {  // lane 0 only; j = next item to load, in order
+        const int off = lc * a.chunk;
         const uint32_t bytes = (uint32_t)min(a.chunk, a.row_bytes - off);
         const uint32_t bar = bar0 + 8u * (j % DC_STAGES);
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(smem0 + (uint32_t)((j % DC_STAGES) * a.chunk), a.x + (size_t)t * a.row_bytes + off, bytes, bar);
+        bulk_g2s(smem0 + (uint32_t)((j % DC_STAGES) * a.chunk), a.x + (size_t)lt * a.row_bytes + off, bytes, bar);
     };
-    if (lane == 0)
-        for (int j = 0; j < DC_STAGES - 1 && j < n; ++j) load(j);
+    auto advance = [&]() {
+        if (++lc == a.nchunks) {
+            lc = 0;
+            ++lt;
+        }
+    };
+    for (int j = 0; j < DC_STAGES - 1 && j < n; ++j) {
+        if (lane == 0) load(j);
+        advance();
+    }
     int issued = min(DC_STAGES - 1, n);  // loads issued (lane 0's count, kept uniform)
 
     // Lane k holds the current token's slot k; the next token's is loaded ahead.
@@ -91,9 +100,8 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
     if (n > 0 && lane < a.K) nxt = __ldg(a.slot_of + (size_t)(first / a.nchunks) * a.K + lane);
     bool ok = true;
     int i = 0;
-    for (; i < n; ++i) {
-        const long long item = first + i;
-        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+    int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
+    for (; i < n; ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
         if (t != t_cur) {
             t_cur = t;
             cur = nxt;
@@ -118,6 +126,7 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
             bulk_wait_read<1>();
             __syncwarp();
             if (lane == 0) load(j);
+            advance();
             issued = j + 1;
         }
     }
@@ -132,12 +141,15 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
 // FP8 e4m3, 128-channel blocks
 // ------------------------------------------------------------------------------------------
 
-constexpr int DQ_STAGES = 8;
+constexpr int DQ_MAX_STAGES = 8;
+constexpr int DQ_STAGE_BUDGET = 48 * 1024;                   // bytes of input ring per CTA
 constexpr int DQ_CONSUMER_WARPS = 4;
 constexpr int DQ_CONSUMERS = DQ_CONSUMER_WARPS * 32;
 constexpr int DQ_THREADS = DQ_CONSUMERS + 32;
-constexpr int DQ_UNIT = 16;                                  // channels per consumer thread
-constexpr int DQ_MAX_BLOCKS = DQ_CONSUMERS * DQ_UNIT / 128;  // 128-channel blocks per item
+constexpr int DQ_UNIT = 16;                                  // channels of one thread unit
+constexpr int DQ_UNITS = 2;                                  // units per thread and item
+constexpr int DQ_SPAN = DQ_CONSUMERS * DQ_UNIT;              // channels between a thread's units
+constexpr int DQ_MAX_BLOCKS = DQ_UNITS * DQ_SPAN / 128;      // 128-channel blocks per item
 constexpr int DQ_HDR = 128;                                  // per-stage header: the token's K slots
 
 struct Fp8Args {
@@ -152,7 +164,21 @@ struct Fp8Args {
     int bpc;         // 128-channel blocks per item (the last item of a row may hold fewer)
     int nchunks;     // items per token
     int stage;       // bytes per stage: header + bpc * 128 * esz
+    int stages;      // stages in the ring (<= DQ_MAX_STAGES)
 };
+
+// s = amax / 448 rounded to nearest even.  For amax >= 2^-80 this is
+// Markstein's correction of amax * RN(1/448) (exact there; checked against
+// IEEE division for every bf16 amax and 1.6e7 fp32 ones), else IEEE division.
+__device__ __forceinline__ float scale_of(float amax) {
+    if (amax >= 0x1p-80f) {
+        const float r = 0x1.24924ap-9f;  // RN(1/448)
+        const float q0 = __fmul_rn(amax, r);
+        const float e = __fmaf_rn(-q0, 448.0f, amax);
+        return __fmaf_rn(e, r, q0);
+    }
+    return __fdiv_rn(amax, 448.0f);
+}
 
 // q = x / s rounded to nearest even, for normal x, s: Markstein's correction
 // of x * r with r = 1/s correctly rounded (P. Markstein, "Computation of
@@ -201,19 +227,22 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
     return U4{w[0], w[1], w[2], w[3]};
 }
 
-template <bool IN_F32>
+// KT: K known at compile time (0 = runtime K).
+template <bool IN_F32, int KT>
 __global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    // layout: [DQ_STAGES][header (K slots) | bpc*128*esz input bytes] | barriers
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DQ_STAGES * a.stage);
+    // layout: [stages][header (K slots) | bpc*128*esz input bytes] | barriers
+    const int NS = a.stages;
+    const int K = KT > 0 ? KT : a.K;
     const uint32_t smem0 = smem_addr(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * a.stage);
     const uint32_t bar0 = smem_addr(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (DQ_STAGES + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (DQ_MAX_STAGES + s); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < DQ_STAGES; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), DQ_CONSUMER_WARPS);
         }
@@ -234,13 +263,13 @@ __global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args 
         int t_cur = -1;
         int nxt = -1;
         const int t_first = (int)(first / a.nchunks);
-        if (first < last && lane < a.K) nxt = __ldg(a.slot_of + (size_t)t_first * a.K + lane);
+        if (first < last && lane < K) nxt = __ldg(a.slot_of + (size_t)t_first * K + lane);
         int cur = -1;
         int i = 0;
         bool ok = true;
-        for (long long item = first; item < last && ok; ++item, ++i) {
-            const int s = i % DQ_STAGES;
-            const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
+        int t = t_first, c = (int)(first - (long long)t_first * a.nchunks);
+        for (long long item = first; item < last && ok; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
+            const int s = i % NS;
             if (t != t_cur) {
                 t_cur = t;
                 cur = nxt;
@@ -249,15 +278,15 @@ __global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args 
                     cur = -1;
                 }
                 const int tn = t + 1;
-                if (lane < a.K && (long long)tn * a.nchunks < last) nxt = __ldg(a.slot_of + (size_t)tn * a.K + lane);
+                if (lane < K && (long long)tn * a.nchunks < last) nxt = __ldg(a.slot_of + (size_t)tn * K + lane);
             }
-            if (i >= DQ_STAGES)
-                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / DQ_STAGES) - 1) & 1, a.status));
+            if (i >= NS)
+                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / NS) - 1) & 1, a.status));
             if (!ok) break;
             const int off = c * chunk_bytes;
             const uint32_t bytes = (uint32_t)min(chunk_bytes, row_bytes - off);
             const uint32_t st = smem0 + (uint32_t)(s * a.stage);
-            if (lane < a.K) asm volatile("st.shared.s32 [%0], %1;" ::"r"(st + 4u * lane), "r"(cur) : "memory");
+            if (lane < K) asm volatile("st.shared.s32 [%0], %1;" ::"r"(st + 4u * lane), "r"(cur) : "memory");
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(full_bar(s), bytes);
@@ -265,72 +294,94 @@ __global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args 
             }
         }
         if (lane == 0) {
-            for (int j = i - DQ_STAGES; j < i; ++j)
-                if (j >= 0) mbar_wait(full_bar(j % DQ_STAGES), (j / DQ_STAGES) & 1, a.status);
+            for (int j = i - NS; j < i; ++j)
+                if (j >= 0) mbar_wait(full_bar(j % NS), (j / NS) & 1, a.status);
         }
         return;
     }
 
     // ------------------------------- consumers -------------------------------
-    // Thread tid owns channels [16 tid, 16 tid + 16) of the item; the 8 threads
-    // of a 128-channel block reduce its amax.  Codes: one 16-byte store per copy.
+    // Thread tid owns two 16-channel units of the item, channels
+    // [16 tid + 2048 u, +16) for u = 0, 1 (two independent chains); the 8
+    // threads of a 128-channel block reduce its amax.  Codes: one 16-byte store
+    // per unit and copy (a warp writes 512 contiguous bytes per copy); the
+    // block's lead thread stores the scale.
+    int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
     int i = 0;
-    for (long long item = first; item < last; ++item, ++i) {
-        const int s = i % DQ_STAGES;
-        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / DQ_STAGES) & 1, a.status))) break;
-        const int t = (int)(item / a.nchunks), c = (int)(item - (long long)t * a.nchunks);
-        const int col0 = c * a.bpc * 128;                   // first channel of the item
-        const int nch = min(a.bpc * 128, a.H - col0);       // channels in this item
-        const bool active = tid * DQ_UNIT < nch;            // whole blocks: groups all-or-nothing
+    for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
+        const int s = i % NS;
+        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / NS) & 1, a.status))) break;
+        const int col0 = c * a.bpc * 128;              // first channel of the item
+        const int nch = min(a.bpc * 128, a.H - col0);  // channels in this item
         const uint32_t st = smem0 + (uint32_t)(s * a.stage);
-        float f[16];
-        if (active) {
-            const uint32_t src = st + DQ_HDR + (uint32_t)(tid * DQ_UNIT * a.esz);
-            if (IN_F32) {
+        float f[DQ_UNITS][16];
+        bool active[DQ_UNITS];
 #pragma unroll
-                for (int l = 0; l < 4; ++l) {
-                    const U4 v = lds128(src + 16u * l);
-                    f[4 * l + 0] = __uint_as_float(v.x);
-                    f[4 * l + 1] = __uint_as_float(v.y);
-                    f[4 * l + 2] = __uint_as_float(v.z);
-                    f[4 * l + 3] = __uint_as_float(v.w);
+        for (int u = 0; u < DQ_UNITS; ++u) {
+            const int ch = u * DQ_SPAN + tid * DQ_UNIT;
+            active[u] = ch < nch;  // whole blocks: groups all-or-nothing
+            if (active[u]) {
+                const uint32_t src = st + DQ_HDR + (uint32_t)(ch * a.esz);
+                if (IN_F32) {
+#pragma unroll
+                    for (int l = 0; l < 4; ++l) {
+                        const U4 v = lds128(src + 16u * l);
+                        f[u][4 * l + 0] = __uint_as_float(v.x);
+                        f[u][4 * l + 1] = __uint_as_float(v.y);
+                        f[u][4 * l + 2] = __uint_as_float(v.z);
+                        f[u][4 * l + 3] = __uint_as_float(v.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int l = 0; l < 2; ++l) {
+                        const U4 v = lds128(src + 16u * l);
+                        f[u][8 * l + 0] = bf16lo(v.x); f[u][8 * l + 1] = bf16hi(v.x);
+                        f[u][8 * l + 2] = bf16lo(v.y); f[u][8 * l + 3] = bf16hi(v.y);
+                        f[u][8 * l + 4] = bf16lo(v.z); f[u][8 * l + 5] = bf16hi(v.z);
+                        f[u][8 * l + 6] = bf16lo(v.w); f[u][8 * l + 7] = bf16hi(v.w);
+                    }
                 }
             } else {
 #pragma unroll
-                for (int l = 0; l < 2; ++l) {
-                    const U4 v = lds128(src + 16u * l);
-                    f[8 * l + 0] = bf16lo(v.x); f[8 * l + 1] = bf16hi(v.x);
-                    f[8 * l + 2] = bf16lo(v.y); f[8 * l + 3] = bf16hi(v.y);
-                    f[8 * l + 4] = bf16lo(v.z); f[8 * l + 5] = bf16hi(v.z);
-                    f[8 * l + 6] = bf16lo(v.w); f[8 * l + 7] = bf16hi(v.w);
-                }
+                for (int e = 0; e < 16; ++e) f[u][e] = 0.f;
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = 0.f;
         }
         int myslot = -1;
-        if (lane < a.K) asm volatile("ld.shared.s32 %0, [%1];" : "=r"(myslot) : "r"(st + 4u * lane) : "memory");
+        if (lane < K) asm volatile("ld.shared.s32 %0, [%1];" : "=r"(myslot) : "r"(st + 4u * lane) : "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(s));  // input stage no longer needed
 
-        float amax = 0.f;
+        float scale[DQ_UNITS];
+        U4 q[DQ_UNITS];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 4));
-        const float scale = __fdiv_rn(amax, 448.0f);
-        const U4 q = quant16(f, scale);
+        for (int u = 0; u < DQ_UNITS; ++u) {
+            float amax = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[u][e]));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 4));
+            scale[u] = scale_of(amax);
+            q[u] = quant16(f[u], scale[u]);
+        }
 
-        const int col = col0 + tid * DQ_UNIT;
-        const bool lead = active && (tid & 7) == 0;
-        const int blk = col >> 7;
-        for (int k = 0; k < a.K; ++k) {
+        const bool lead = (lane & 7) == 0;
+        uint8_t *const xcol = a.xd + col0 + tid * DQ_UNIT;
+        float *const scol = a.xs + ((col0 + tid * DQ_UNIT) >> 7);
+        constexpr int KU = KT > 0 ? KT : 1;
+#pragma unroll(KU)
+        for (int k = 0; k < K; ++k) {
             const int sl = __shfl_sync(FULL, myslot, k);
             if (sl < 0) continue;
-            if (active) st_v4(a.xd + (size_t)sl * a.H + col, q);
-            if (lead) a.xs[(size_t)sl * nb + blk] = scale;
+            uint8_t *const row = xcol + (size_t)sl * a.H;
+            float *const srow = scol + (size_t)sl * nb;
+#pragma unroll
+            for (int u = 0; u < DQ_UNITS; ++u) {
+                if (active[u]) {
+                    st_v4(row + u * DQ_SPAN, q[u]);
+                    if (lead) srow[u * (DQ_SPAN >> 7)] = scale[u];
+                }
+            }
         }
     }
 }
@@ -368,26 +419,28 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
         return launch_pdl(dispatch_copy_kernel, dim3(grid), dim3(32), smem, st, a);
     }
     Fp8Args a{reinterpret_cast<const uint8_t *>(x), slot_of, reinterpret_cast<uint8_t *>(xd), xs, status,
-              cap, S, H, K, esz, 0, 0, 0};
+              cap, S, H, K, esz, 0, 0, 0, 0};
     // Split each row into the fewest items of at most DQ_MAX_BLOCKS blocks, as evenly as possible.
     const int blocks = H / 128;
     const int n = (blocks + DQ_MAX_BLOCKS - 1) / DQ_MAX_BLOCKS;
     a.bpc = (blocks + n - 1) / n;
     a.nchunks = (blocks + a.bpc - 1) / a.bpc;
     a.stage = DQ_HDR + a.bpc * 128 * esz;
-    const size_t smem = (size_t)DQ_STAGES * a.stage + 2 * DQ_STAGES * 8;
-    unsigned grid = 1;
-    cudaError_t e;
-    if (dtype == MOE_DTYPE_BF16) {
-        static KernelSlots<decltype(&dispatch_fp8_kernel<false>)> slots;
-        e = persistent_grid(slots, &dispatch_fp8_kernel<false>, DQ_THREADS, smem, (long long)S * a.nchunks, &grid);
+    a.stages = DQ_STAGE_BUDGET / a.stage;
+    if (a.stages > DQ_MAX_STAGES) a.stages = DQ_MAX_STAGES;
+    if (a.stages < 3) a.stages = 3;
+    const size_t smem = (size_t)a.stages * a.stage + 2 * DQ_MAX_STAGES * 8;
+    const long long nitems = (long long)S * a.nchunks;
+    auto go = [&](auto kern) -> cudaError_t {
+        static KernelSlots<decltype(kern)> slots;
+        unsigned grid = 1;
+        cudaError_t e = persistent_grid(slots, kern, DQ_THREADS, smem, nitems, &grid);
         if (e != cudaSuccess) return e;
-        return launch_pdl(dispatch_fp8_kernel<false>, dim3(grid), dim3(DQ_THREADS), smem, st, a);
-    }
-    static KernelSlots<decltype(&dispatch_fp8_kernel<true>)> slots;
-    e = persistent_grid(slots, &dispatch_fp8_kernel<true>, DQ_THREADS, smem, (long long)S * a.nchunks, &grid);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(dispatch_fp8_kernel<true>, dim3(grid), dim3(DQ_THREADS), smem, st, a);
+        return launch_pdl(kern, dim3(grid), dim3(DQ_THREADS), smem, st, a);
+    };
+    if (dtype == MOE_DTYPE_BF16)
+        return K == 8 ? go(&dispatch_fp8_kernel<false, 8>) : go(&dispatch_fp8_kernel<false, 0>);
+    return K == 8 ? go(&dispatch_fp8_kernel<true, 8>) : go(&dispatch_fp8_kernel<true, 0>);
 }
 
 }  // namespace moe

@@ -254,7 +254,14 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
     const size_t smem = (size_t)LT_WARPS * E * sizeof(uint16_t);
-    cudaError_t err = launch_pdl(layout_hist_kernel, dim3(T), dim3(LT_THREADS), smem, st, topk_idx, npairs,
+    static KernelSlots<decltype(&layout_hist_kernel)> hist_slots;
+    static KernelSlots<decltype(&layout_slots_kernel)> slot_slots;
+    int n_sms = 0, per_sm = 0;
+    cudaError_t err = hist_slots.prepare(&layout_hist_kernel, LT_THREADS, smem, &n_sms, &per_sm);
+    if (err != cudaSuccess) return err;
+    err = slot_slots.prepare(&layout_slots_kernel, LT_THREADS, smem, &n_sms, &per_sm);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(layout_hist_kernel, dim3(T), dim3(LT_THREADS), smem, st, topk_idx, npairs,
                                  E, R, P, cap, hist, hdr, counts, offsets, rank_offsets, status);
     if (err != cudaSuccess) return err;
     return launch_pdl(layout_slots_kernel, dim3(T), dim3(LT_THREADS), smem, st, topk_idx, npairs, E,

@@ -81,6 +81,10 @@ static cudaError_t launch_route(const float *logits, int S, int E, int K, int32_
     const int cap_blocks = sms * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
     if (blocks < 1) blocks = 1;
+    static KernelSlots<decltype(&route_topk_kernel<NPER>)> slots;
+    int n_sms = 0, per_sm = 0;
+    const cudaError_t e = slots.prepare(&route_topk_kernel<NPER>, threads, 0, &n_sms, &per_sm);
+    if (e != cudaSuccess) return e;
     return launch_pdl(route_topk_kernel<NPER>, dim3(blocks), dim3(threads), 0, st, logits, S, E, K, idx, w);
 }
 
