@@ -135,8 +135,8 @@ def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, token_padding: i
     """Histogram + prefix scan into the padded expert-contiguous layout.
 
     ``workspace`` (uint8, >= moe_dispatch_layout_workspace bytes) must be zero-filled
-    before its first use; each call leaves it zeroed.  A fresh zeroed one is
-    allocated when it is not given.  ``out`` may carry a Layout to write into."""
+    before its first use; each call leaves it ready for the next.  A fresh zeroed
+    one is allocated when it is not given.  ``out`` may carry a Layout to write into."""
     _dev(topk_idx, "topk_idx", (torch.int32,))
     S, K = topk_idx.shape
     dev = topk_idx.device

@@ -137,7 +137,10 @@ class MoeBuffer:
         return self.combine(y, shared_out, residual, stream=stream)
 
     def read_status(self) -> int:
-        """Reads and clears the device status word (synchronises)."""
+        """Reads and clears the device status word (synchronises).  After a
+        timeout the layout workspace header is zeroed again, as its contract asks."""
         v = int(self.status.item())
         self.status.zero_()
+        if v & B.MOE_STATUS_TIMEOUT:
+            self.workspace[:256].zero_()
         return v

@@ -95,22 +95,42 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Per-kernel launch facts, computed once per (device, dynamic shared memory
-// size): opts the kernel in to that much dynamic shared memory and records
-// how many CTAs of it fit on one SM.  A handful of sizes per kernel are cached;
-// beyond that the query simply runs again.  Races between host threads only
-// repeat idempotent driver calls.
+// size): how many CTAs of that size fit on one SM.  The kernel's opt-in limit
+// for dynamic shared memory is one setting per device that the last call
+// wins, so it is only ever raised, to the largest size requested so far, and
+// every smaller launch stays within it.  A handful of sizes per kernel are
+// cached; beyond that the query simply runs again.  Races between host
+// threads only repeat idempotent driver calls.
 template <typename Kern>
 struct KernelSlots {
     static constexpr int N = 8;
+    static constexpr int MAXDEV = 64;
     int dev[N] = {-1, -1, -1, -1, -1, -1, -1, -1};
     size_t smem[N] = {};
     int sms[N] = {}, per_sm[N] = {};
     int next = 0;
+    size_t limit_set[MAXDEV] = {};
+    bool carveout_set[MAXDEV] = {};
 
     cudaError_t prepare(Kern kern, int threads, size_t bytes, int *n_sms, int *n_per_sm) {
         int d = 0;
         cudaError_t e = cudaGetDevice(&d);
         if (e != cudaSuccess) return e;
+        if (d < 0 || d >= MAXDEV) return cudaErrorInvalidDevice;
+        if (bytes > limit_set[d]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+            if (e != cudaSuccess) return e;
+            limit_set[d] = bytes;
+        }
+        if (!carveout_set[d]) {
+            // Every kernel of the library asks for the largest shared-memory
+            // carveout, so consecutive kernels never wait for an L1/shared
+            // split to be reconfigured.
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+            carveout_set[d] = true;
+        }
         for (int i = 0; i < N; ++i) {
             if (dev[i] == d && smem[i] == bytes) {
                 *n_sms = sms[i];
@@ -118,16 +138,6 @@ struct KernelSlots {
                 return cudaSuccess;
             }
         }
-        if (bytes > 48 * 1024) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-            if (e != cudaSuccess) return e;
-        }
-        // Every kernel of the library asks for the largest shared-memory
-        // carveout, so consecutive kernels never wait for an L1/shared split
-        // to be reconfigured.
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
         int s = 0, p = 0;
         e = cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, d);
         if (e != cudaSuccess) return e;

@@ -7,7 +7,11 @@
 // and Dispatch (tokens of one expert contiguous; the source of each row kept
 // for the combine).
 //
-// Two kernels, no spin-waits and no global atomics except one arrival counter:
+// Layouts whose tile histograms every CTA can scan (T * E <= 64 Ki entries) and
+// whose tiles fit one co-resident grid run as ONE cooperative kernel
+// (layout_fused, below): ranks in registers, one bounded grid barrier, each CTA
+// scanning the tile histograms itself.  Larger layouts use two kernels, with no
+// spin-waits and no global atomics except one arrival counter:
 //
 //  layout_hist   one CTA per tile of LT_TILE pairs.  Each warp ranks its 32
 //                pairs by expert with __match_any_sync (peers share an expert;
@@ -27,11 +31,14 @@
 // (ascending t*K + k) with the same expert: a stable counting sort.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
 struct LayoutHeader {
-    unsigned int ticket;
+    unsigned int ticket;   // two-kernel path: arrival ticket, reset by the last CTA
+    unsigned int count;    // fused path: grid-barrier arrivals, reset by the last arriver
+    unsigned int gen;      // fused path: grid-barrier generation (only ever incremented)
 };
 
 __device__ __forceinline__ int pad_count(int c, int P) { return P > 0 ? ((c + P - 1) / P) * P : c; }
@@ -56,16 +63,19 @@ __global__ void __launch_bounds__(LT_THREADS)
     __syncthreads();
 
     bool bad = false;
+    int ev[LT_ITEMS];  // all loads first, so their latencies overlap
 #pragma unroll
     for (int it = 0; it < LT_ITEMS; ++it) {
         const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
-        int e = -1;
-        if (p < npairs) {
-            e = __ldg(topk_idx + p);
-            if (e < 0 || e >= E) {
-                bad = true;
-                e = -1;
-            }
+        ev[it] = p < npairs ? __ldg(topk_idx + p) : -1;
+    }
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        int e = ev[it];
+        if (p < npairs && (e < 0 || e >= E)) {
+            bad = true;
+            e = -1;
         }
         const unsigned peers = __match_any_sync(FULL, e);
         if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] += (uint16_t)__popc(peers);
@@ -96,7 +106,13 @@ __global__ void __launch_bounds__(LT_THREADS)
         const int g = idx / E, e = idx - g * E;
         const int t1 = min(T, (g + 1) * tpg);
         int c = 0;
-        for (int t = g * tpg; t < t1; ++t) c += __ldcg(hist + (size_t)t * E + e);
+        for (int t = g * tpg; t < t1; t += 8) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = t + j < t1 ? __ldcg(hist + (size_t)(t + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c += v[j];
+        }
         s_part[idx] = c;
     }
     __syncthreads();
@@ -179,14 +195,16 @@ __global__ void __launch_bounds__(LT_THREADS)
     // through L2 (ld.global.cg), never a stale L1 line.
     int my_e[LT_ITEMS], my_r[LT_ITEMS];
     const unsigned lt = lanemask_lt();
+    int ev[LT_ITEMS];  // all loads first, so their latencies overlap
 #pragma unroll
     for (int it = 0; it < LT_ITEMS; ++it) {
         const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
-        int e = -1;
-        if (p < npairs) {
-            e = __ldcg(topk_idx + p);
-            if (e < 0 || e >= E) e = -1;
-        }
+        ev[it] = p < npairs ? __ldcg(topk_idx + p) : -1;
+    }
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        int e = ev[it];
+        if (e < 0 || e >= E) e = -1;
         const unsigned peers = __match_any_sync(FULL, e);
         const int before = e >= 0 ? (int)whist[w * E + e] : 0;
         __syncwarp();
@@ -245,6 +263,287 @@ __global__ void __launch_bounds__(LT_THREADS)
         row_src[r] = -1;
 }
 
+// ------------------------------------------------------------------------------------------
+// Fused single-launch layout (cooperative grid; used when every CTA can read
+// all tile histograms cheaply): phase 1 ranks the pairs of this CTA's tiles
+// and publishes the tile histograms; one grid barrier; phase 2 has every CTA
+// scan the tile histograms itself (its tiles' prefixes, the totals, the padded
+// offsets) and write its slots.  The barrier's wait is time-bounded.
+// ------------------------------------------------------------------------------------------
+
+constexpr int LF_MAX_HIST = 64 * 1024;  // T * E entries a CTA may scan in phase 2
+
+// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  Sense
+// reversal: read the generation, arrive; the last arriver resets the count and
+// bumps the generation; the others wait (bounded) for the bump.  False on timeout.
+__device__ bool grid_barrier(LayoutHeader *hdr, int32_t *status) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        const unsigned gen = *(volatile unsigned *)&hdr->gen;
+        __threadfence();
+        const unsigned prev = atomicAdd(&hdr->count, 1u);
+        if (prev == gridDim.x - 1) {
+            *(volatile unsigned *)&hdr->count = 0u;
+            __threadfence();
+            atomicExch(&hdr->gen, gen + 1u);
+        } else {
+            const unsigned long long t0 = globaltimer();
+            while (*(volatile unsigned *)&hdr->gen == gen) {
+                if (globaltimer() - t0 > MOE_WAIT_NS) {
+                    set_status(status, MOE_STATUS_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+// Ranks the 32 * LT_ITEMS pairs of warp w in tile `tile` by expert: my_e = expert
+// (-1: none or invalid), my_r = rank among the warp's earlier pairs of that expert;
+// whist[w][e] accumulates the warp's counts (whist must be zeroed).
+__device__ __forceinline__ bool rank_tile(const int32_t *topk_idx, int npairs, int E, int tile, int w, int lane,
+                                          uint16_t *whist, int (&my_e)[LT_ITEMS], int (&my_r)[LT_ITEMS]) {
+    bool bad = false;
+    const unsigned lt = lanemask_lt();
+    int ev[LT_ITEMS];  // all loads first, so their latencies overlap
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        ev[it] = p < npairs ? __ldcg(topk_idx + p) : -1;
+    }
+#pragma unroll
+    for (int it = 0; it < LT_ITEMS; ++it) {
+        const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+        int e = ev[it];
+        if (p < npairs && (e < 0 || e >= E)) {
+            bad = true;
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(FULL, e);
+        const int before = e >= 0 ? (int)whist[w * E + e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
+        __syncwarp();
+        my_e[it] = e;
+        my_r[it] = before + __popc(peers & lt);
+    }
+    return bad;
+}
+
+__global__ void __launch_bounds__(LT_THREADS)
+    layout_fused_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P, int64_t cap,
+                        int T, int32_t *hist, LayoutHeader *hdr, int32_t *__restrict__ counts,
+                        int32_t *__restrict__ offsets, int32_t *__restrict__ rank_offsets,
+                        int32_t *__restrict__ slot_of, int32_t *__restrict__ row_src, int32_t *status) {
+    extern __shared__ __align__(16) uint8_t lf_smem[];
+    uint16_t *whist = reinterpret_cast<uint16_t *>(lf_smem);                     // [LT_WARPS][E]
+    int *s_all = reinterpret_cast<int *>(lf_smem + ((LT_WARPS * E * 2 + 15) & ~15));  // [G][E]
+    int *s_below = s_all + 1024;                                                  // [G][E]
+    __shared__ int s_tot[1024];
+    __shared__ int s_base[1024];
+    __shared__ int s_off[1025];
+    __shared__ int s_wsum[LT_WARPS];
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    // this CTA's tiles [t0, t1): a contiguous, balanced share of the T tiles
+    const int t0 = (int)((long long)T * blockIdx.x / gridDim.x);
+    const int t1 = (int)((long long)T * (blockIdx.x + 1) / gridDim.x);
+    const bool single = t1 - t0 == 1;
+    pdl_wait();
+    pdl_trigger();
+
+    // ---- phase 1: tile histograms ----
+    int my_e[LT_ITEMS], my_r[LT_ITEMS];
+    bool bad = false;
+    for (int tile = t0; tile < t1; ++tile) {
+        for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
+        __syncthreads();
+        bad |= rank_tile(topk_idx, npairs, E, tile, w, lane, whist, my_e, my_r);
+        __syncthreads();
+        for (int e = tid; e < E; e += LT_THREADS) {
+            int cnt = 0;
+#pragma unroll
+            for (int ww = 0; ww < LT_WARPS; ++ww) cnt += whist[ww * E + e];
+            hist[(size_t)tile * E + e] = cnt;
+        }
+        if (!single) __syncthreads();  // whist is rebuilt for the next tile
+    }
+    if (bad) set_status(status, MOE_STATUS_BAD_INDEX);
+    __threadfence();
+    if (!grid_barrier(hdr, status)) return;
+
+    // ---- phase 2a: per expert, the sum over tiles below t0 and over all tiles ----
+    int G = LT_THREADS / E;
+    if (G < 1) G = 1;
+    if (G > T) G = T;
+    const int tpg = (T + G - 1) / G;
+    for (int idx = tid; idx < G * E; idx += LT_THREADS) {
+        const int g = idx / E, e = idx - g * E;
+        const int ta = g * tpg, tb = min(T, ta + tpg);
+        int all = 0, below = 0;
+        for (int tt = ta; tt < tb; tt += 8) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = tt + j < tb ? __ldcg(hist + (size_t)(tt + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                all += v[j];
+                below += tt + j < t0 ? v[j] : 0;
+            }
+        }
+        s_all[idx] = all;
+        s_below[idx] = below;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += LT_THREADS) {
+        int all = 0, below = 0;
+        for (int g = 0; g < G; ++g) {
+            all += s_all[g * E + e];
+            below += s_below[g * E + e];
+        }
+        s_tot[e] = all;
+        s_base[e] = below;
+    }
+    __syncthreads();
+    // ---- phase 2b: exclusive scan of the padded counts over experts, two per thread ----
+    const int e0 = 2 * tid, e1 = 2 * tid + 1;
+    const int p0 = e0 < E ? pad_count(s_tot[e0], P) : 0;
+    const int p1 = e1 < E ? pad_count(s_tot[e1], P) : 0;
+    int incl = p0 + p1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = lane < LT_WARPS ? s_wsum[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(FULL, v, off);
+            if (lane >= off) v += o;
+        }
+        if (lane < LT_WARPS) s_wsum[lane] = v;
+    }
+    __syncthreads();
+    const int base = incl - (p0 + p1) + (w > 0 ? s_wsum[w - 1] : 0);
+    if (e0 < E) s_off[e0] = base;
+    if (e1 < E) s_off[e1] = base + p0;
+    if (tid == 0) s_off[E] = s_wsum[LT_WARPS - 1];
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int e = tid; e <= E; e += LT_THREADS) offsets[e] = s_off[e];
+        for (int e = tid; e < E; e += LT_THREADS) counts[e] = s_tot[e];
+        const int Eloc = E / R;
+        for (int r = tid; r <= R; r += LT_THREADS) rank_offsets[r] = s_off[r * Eloc];
+        if (tid == 0 && (int64_t)s_off[E] > cap) set_status(status, MOE_STATUS_OVERFLOW);
+    }
+
+    // ---- phase 2c: slots of this CTA's tiles ----
+    bool over = false;
+    for (int tile = t0; tile < t1; ++tile) {
+        if (!single) {
+            for (int i = tid; i < LT_WARPS * E; i += LT_THREADS) whist[i] = 0;
+            __syncthreads();
+            rank_tile(topk_idx, npairs, E, tile, w, lane, whist, my_e, my_r);
+            __syncthreads();
+        }
+        // per-warp counts -> exclusive prefix over warps; the tile total moves the base on
+        for (int e = tid; e < E; e += LT_THREADS) {
+            int run = 0;
+#pragma unroll
+            for (int ww = 0; ww < LT_WARPS; ++ww) {
+                const int cnt = whist[ww * E + e];
+                whist[ww * E + e] = (uint16_t)run;
+                run += cnt;
+            }
+            s_all[e] = s_off[e] + s_base[e];  // first row of this tile's pairs of expert e
+            s_base[e] += run;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int it = 0; it < LT_ITEMS; ++it) {
+            const int p = tile * LT_TILE + (w * LT_ITEMS + it) * 32 + lane;
+            if (p >= npairs) continue;
+            const int e = my_e[it];
+            int sl = -1;
+            if (e >= 0) {
+                sl = s_all[e] + whist[w * E + e] + my_r[it];
+                if ((int64_t)sl >= cap) {
+                    sl = -1;
+                    over = true;
+                }
+            }
+            slot_of[p] = sl;
+            if (sl >= 0) row_src[sl] = p;
+        }
+        __syncthreads();
+    }
+    if (over) set_status(status, MOE_STATUS_OVERFLOW);
+
+    // ---- padding rows (one warp per expert) and rows past the layout ----
+    const int gw = blockIdx.x * LT_WARPS + w, nw = gridDim.x * LT_WARPS;
+    for (int e = gw; e < E; e += nw) {
+        const int64_t lo = (int64_t)s_off[e] + s_tot[e];
+        int64_t hi = s_off[e + 1];
+        if (hi > cap) hi = cap;
+        for (int64_t r = lo + lane; r < hi; r += 32) row_src[r] = -1;
+    }
+    for (int64_t r = (int64_t)s_off[E] + (int64_t)blockIdx.x * LT_THREADS + tid; r < cap;
+         r += (int64_t)gridDim.x * LT_THREADS)
+        row_src[r] = -1;
+}
+
+static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap, int T,
+                                       int32_t *hist, LayoutHeader *hdr, int32_t *counts, int32_t *offsets,
+                                       int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src, int32_t *status,
+                                       cudaStream_t st, bool *launched) {
+    *launched = false;
+    const size_t smem = (size_t)((LT_WARPS * E * 2 + 15) & ~15) + 2 * 1024 * sizeof(int);
+    static KernelSlots<decltype(&layout_fused_kernel)> slots;
+    int sms = 0, per_sm = 0;
+    cudaError_t e = slots.prepare(&layout_fused_kernel, LT_THREADS, smem, &sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    long long grid = (long long)sms * per_sm;  // all CTAs must be co-resident
+    if (grid > T) grid = T;
+    if (grid < 1 || (long long)T * E > LF_MAX_HIST) return cudaSuccess;  // not launched: use two kernels
+    // Cooperative (all CTAs co-resident, for the grid barrier) and, where the
+    // driver accepts the pair, programmatic serialisation too (see pdl_wait).
+    static int pdl_ok = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(LT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_ok ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts,
+                           offsets, rank_offsets, slot_of, row_src, status);
+    if (e != cudaSuccess && pdl_ok) {
+        (void)cudaGetLastError();  // the pair was refused: launch cooperative only from now on
+        pdl_ok = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts,
+                               offsets, rank_offsets, slot_of, row_src, status);
+    }
+    if (e == cudaSuccess) *launched = true;
+    return e;
+}
+
 cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int P,
                           int32_t *counts, int32_t *offsets, int32_t *rank_offsets,
                           int32_t *slot_of, int32_t *row_src, int64_t cap, void *workspace,
@@ -253,6 +552,11 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     const int T = layout_tiles(npairs);
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
+    bool launched = false;
+    cudaError_t fe = launch_layout_fused(topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts, offsets,
+                                         rank_offsets, slot_of, row_src, status, st, &launched);
+    if (fe != cudaSuccess) return fe;
+    if (launched) return cudaSuccess;
     const size_t smem = (size_t)LT_WARPS * E * sizeof(uint16_t);
     static KernelSlots<decltype(&layout_hist_kernel)> hist_slots;
     static KernelSlots<decltype(&layout_slots_kernel)> slot_slots;

@@ -137,10 +137,13 @@ MOE_API size_t moe_dispatch_layout_workspace(int S, int E, int K);
  * pair order makes the layout deterministic.
  *
  * workspace: device scratch of at least moe_dispatch_layout_workspace(S,E,K)
- *   bytes, 256-byte aligned, owned by the caller.  Its first 256 bytes must be
- *   zero before the first call; every call leaves them zero again, so one
- *   zero-filled workspace can serve any number of calls on one stream.  Calls
- *   that may run concurrently need separate workspaces.
+ *   bytes, 256-byte aligned, owned by the caller.  Its first 256 bytes (the
+ *   grid-synchronisation header) must be zero before the first call; every
+ *   call that completes leaves them ready for the next one, so one zero-filled
+ *   workspace serves any number of calls on one stream, whatever their sizes.
+ *   Do not modify it between calls.  After a call that reported
+ *   MOE_STATUS_TIMEOUT, zero the header again.  Calls that may run
+ *   concurrently need separate workspaces.
  * Device status: MOE_STATUS_BAD_INDEX (pair dropped, not counted),
  *   MOE_STATUS_OVERFLOW (offsets[E] > cap; pairs whose slot would be >= cap
  *   get slot_of = -1).
