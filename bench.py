@@ -285,6 +285,21 @@ def run_ours(args, w, rank, world, local_rank):
     if buf.read_status() != 0:
         raise RuntimeError("device status flagged a problem during warm-up")
 
+    graph = None
+    if args.graph:
+        graph = buf.capture(d["logits"], d["x"], d["y"], sh, rs)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        if buf.read_status() != 0:
+            raise RuntimeError("device status flagged a problem in the captured step")
+
+    def one_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            buf.step(d["logits"], d["x"], d["y"], sh, rs)
+
     # ---- timed region 1 (value): K steps back to back, events only at the ends, so
     # consecutive kernels overlap through programmatic dependent launch ----
     K = args.steps
@@ -296,7 +311,7 @@ def run_ours(args, w, rank, world, local_rank):
     t_start.record()
     h0 = time.perf_counter()
     for _ in range(K):
-        buf.step(d["logits"], d["x"], d["y"], sh, rs)
+        one_step()
     t_end.record()
     host_us = (time.perf_counter() - h0) / K * 1e6
     torch.cuda.synchronize()
@@ -392,8 +407,9 @@ def run_ours(args, w, rank, world, local_rank):
                              "frac_of_peak": dc_gbs / peak, "frac_of_nominal_8tbs": dc_gbs / 8000.0},
         "phases": phases, "roofline": roofline, "e2e": e2e,
         "gpu_launches": K * buf.KERNELS_PER_STEP, "clocks": clocks,
-        "timing": "value: K steps back to back (events at the ends only); phases/roofline: a second "
-                  "pass of K steps with an event between kernels",
+        "timing": "value: K steps back to back (events at the ends only)"
+                  + (", each step one CUDA-graph replay" if graph is not None else ", eager calls")
+                  + "; phases/roofline: a second pass of K eager steps with an event between kernels",
         "host_enqueue_us_per_step": host_us,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -411,6 +427,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="time the value pass as CUDA-graph replays of one step (default; "
+                         "--no-graph times eager calls)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override S (a smaller case of the same workload, for profiling)")
     args = ap.parse_args(argv)

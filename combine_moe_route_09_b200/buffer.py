@@ -136,6 +136,16 @@ class MoeBuffer:
         self.dispatch(x, stream)
         return self.combine(y, shared_out, residual, stream=stream)
 
+    def capture(self, logits, x, y, shared_out=None, residual=None):
+        """Records one step into a CUDA graph and returns it (``graph.replay()``
+        reruns the step).  The graph reads the given input tensors and writes this
+        buffer's outputs at fixed addresses: refill the inputs in place between
+        replays.  Run one eager step first (kernel attributes are set on first use)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step(logits, x, y, shared_out, residual)
+        return g
+
     def read_status(self) -> int:
         """Reads and clears the device status word (synchronises).  After a
         timeout the layout workspace header is zeroed again, as its contract asks."""

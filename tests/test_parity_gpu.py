@@ -132,3 +132,28 @@ def test_full_pass_as_benchmarked(case):
             assert_act_close(host(buf.out_no_routed), ref["rnr"], "residual_no_routed_out")
         assert buf.read_status() == 0
     assert int(buf.workspace[:8].sum().item()) == 0  # arrival ticket and barrier count back at zero
+
+
+def test_captured_step_replays_the_pass(case):
+    """One step captured in a CUDA graph and replayed twice gives the oracle's pass."""
+    w, inp, ref = case
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8")
+    args = [dev(inp["logits"]), dev(inp["x"]), dev(inp["y"])]
+    if w.fused:
+        args += [dev(inp["shared"]), dev(inp["residual"])]
+    buf.step(*args)
+    torch.cuda.synchronize()
+    graph = buf.capture(*args)
+    weight_slack = 2e-5 * abs_weighted_sum(inp["y"], ref["lay"]["slot_of"], ref["w"])
+    for _ in range(2):
+        buf.out.zero_()
+        buf.layout.slot_of.fill_(-7)
+        graph.replay()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(buf.topk_idx), ref["idx"])
+        _check_layout(buf.layout, ref["lay"])
+        valid = ref["lay"]["row_src"] >= 0
+        np.testing.assert_array_equal(host(buf.xd)[valid], ref["xd"][valid])
+        assert_act_close(host(buf.out), ref["out"], "residual_out", extra_abs=weight_slack)
+        assert buf.read_status() == 0
