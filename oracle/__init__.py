@@ -51,6 +51,9 @@ def _load():
         lib.oracle_layout.argtypes = [P, I, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch.argtypes = [P, I, I, I, I, P, I, L, P, P]
         lib.oracle_combine.argtypes = [P, I, I, I, I, L, P, P, P, P, P, P]
+        lib.oracle_combine_backward.argtypes = [P, P, P, I, I, I, I, L, P, P, P, P, P]
+        lib.oracle_dispatch_backward.argtypes = [P, I, I, I, I, L, P, P]
+        lib.oracle_route_backward.argtypes = [P, P, P, I, I, I, P]
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -168,6 +171,59 @@ def combine(y: np.ndarray, slot_of: np.ndarray, topk_w: np.ndarray, shared=None,
     if rc:
         raise OracleError("oracle_combine", rc)
     return out, rnr
+
+
+def combine_backward(g, y, slot_of, topk_w, gn=None, grad_y=None, want_skip=True):
+    """Backward of combine: (grad_y [cap,H], grad_w [S,K] fp32, grad_skip [S,H] or None).
+
+    grad_y rows that no pair maps to keep what ``grad_y`` held (zeros if not given)."""
+    g = np.ascontiguousarray(g)
+    y = np.ascontiguousarray(y)
+    slot_of = _c(slot_of, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    S, K = slot_of.shape
+    cap, H = y.shape
+    assert g.dtype == y.dtype and g.shape == (S, H)
+    if gn is not None:
+        gn = np.ascontiguousarray(gn)
+        assert gn.dtype == y.dtype and gn.shape == (S, H)
+    if grad_y is None:
+        grad_y = np.zeros((cap, H), y.dtype)
+    grad_w = np.empty((S, K), np.float32)
+    skip = np.empty((S, H), y.dtype) if want_skip else None
+    rc = _load().oracle_combine_backward(_ptr(g), _ptr(gn), _ptr(y), _dtype_code(y), S, H, K, cap,
+                                         _ptr(slot_of), _ptr(topk_w), _ptr(grad_y), _ptr(grad_w),
+                                         _ptr(skip))
+    if rc:
+        raise OracleError("oracle_combine_backward", rc)
+    return grad_y, grad_w, skip
+
+
+def dispatch_backward(grad_xd, slot_of, S=None):
+    """Backward of the plain dispatch: grad_x [S,H] = sum of the K copies' gradients."""
+    grad_xd = np.ascontiguousarray(grad_xd)
+    slot_of = _c(slot_of, np.int32)
+    S, K = slot_of.shape
+    cap, H = grad_xd.shape
+    grad_x = np.empty((S, H), grad_xd.dtype)
+    rc = _load().oracle_dispatch_backward(_ptr(grad_xd), _dtype_code(grad_xd), S, H, K, cap,
+                                          _ptr(slot_of), _ptr(grad_x))
+    if rc:
+        raise OracleError("oracle_dispatch_backward", rc)
+    return grad_x
+
+
+def route_backward(topk_idx, topk_w, grad_w, E: int):
+    """Backward of the gating softmax: grad_logits [S,E] fp32."""
+    topk_idx = _c(topk_idx, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    grad_w = _c(grad_w, np.float32)
+    S, K = topk_idx.shape
+    out = np.empty((S, E), np.float32)
+    rc = _load().oracle_route_backward(_ptr(topk_idx), _ptr(topk_w), _ptr(grad_w), S, E, K, _ptr(out))
+    if rc:
+        raise OracleError("oracle_route_backward", rc)
+    return out
 
 
 def e4m3_encode(v: float) -> int:

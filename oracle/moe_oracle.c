@@ -13,6 +13,8 @@
  *   oracle_layout       per-expert counts, padded offsets, slot assignment
  *   oracle_dispatch     scatter of token rows (optionally FP8 e4m3, 128-ch blocks)
  *   oracle_combine      gather + top-K weighted sum + dual-residual epilogue
+ *   oracle_combine_backward / oracle_dispatch_backward / oracle_route_backward
+ *                       the transposes of the steps (training)
  *   oracle_e4m3_encode / oracle_e4m3_decode / oracle_bf16_round   format helpers
  *
  * Sources (page title, section):
@@ -380,4 +382,112 @@ int oracle_combine(const void *y, int dtype, int S, int H, int K, int64_t cap,
         }
     }
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the path (training): the transposes of the steps above        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Backward of oracle_combine.  "MoonEP developer guide", core API example:
+ * the backward pass reuses the plan (dispatch of grad_output, combine of the
+ * expert gradients).  With g = dL/d(residual_out) and gn = dL/d(residual_no_routed)
+ * (zero if not given), the forward out = residual + (shared + sum_k w_k y_k),
+ * rnr = residual + shared gives, per token t and pair k with a valid slot:
+ *     grad_y[slot, h]  = w[t,k] * g[t,h]          (fp32 product, rounded once)
+ *     grad_w[t, k]     = sum_h y[slot, h] * g[t,h] (fp64, rounded once to fp32)
+ *     grad_skip[t, h]  = g[t,h] + gn[t,h]         (fp32, rounded once) -- the
+ *                        gradient of both `residual` and `shared_out`
+ * grad_w is 0 for skipped pairs; rows of grad_y no pair maps to are untouched.
+ */
+int oracle_combine_backward(const void *g, const void *gn, const void *y, int dtype, int S, int H,
+                            int K, int64_t cap, const int32_t *slot_of, const float *topk_w,
+                            void *grad_y, float *grad_w, void *grad_skip)
+{
+    if (S < 0 || H < 1 || K < 1) return ORACLE_EINVAL;
+    if (dtype != ORACLE_DTYPE_F32 && dtype != ORACLE_DTYPE_BF16) return ORACLE_EINVAL;
+    int f32 = dtype == ORACLE_DTYPE_F32;
+#define LD(p, i) (f32 ? ((const float *)(p))[i] : bf16_to_f32(((const uint16_t *)(p))[i]))
+    for (int t = 0; t < S; ++t) {
+        for (int k = 0; k < K; ++k) {
+            int32_t s = slot_of[(size_t)t * K + k];
+            double dot = 0.0;
+            if (s >= 0 && (int64_t)s < cap) {
+                float w = topk_w[(size_t)t * K + k];
+                for (int h = 0; h < H; ++h) {
+                    float gv = LD(g, (size_t)t * H + h);
+                    float prod = w * gv;
+                    if (f32) ((float *)grad_y)[(size_t)s * H + h] = prod;
+                    else ((uint16_t *)grad_y)[(size_t)s * H + h] = oracle_bf16_round(prod);
+                    dot += (double)LD(y, (size_t)s * H + h) * (double)gv;
+                }
+            }
+            grad_w[(size_t)t * K + k] = (float)dot;
+        }
+        if (grad_skip) {
+            for (int h = 0; h < H; ++h) {
+                size_t i = (size_t)t * H + h;
+                float v = gn ? LD(g, i) + LD(gn, i) : LD(g, i);
+                if (f32) ((float *)grad_skip)[i] = v;
+                else ((uint16_t *)grad_skip)[i] = oracle_bf16_round(v);
+            }
+        }
+    }
+#undef LD
+    return ORACLE_OK;
+}
+
+/*
+ * Backward of oracle_dispatch (the plain copy; for the FP8 dispatch the
+ * quantiser is passed straight through): every copy of token t received x[t],
+ * so grad_x[t, h] = sum over k with a valid slot of grad_xd[slot, h], summed in
+ * fp32 in ascending k and rounded once (zero when no copy is valid).
+ */
+int oracle_dispatch_backward(const void *grad_xd, int dtype, int S, int H, int K, int64_t cap,
+                             const int32_t *slot_of, void *grad_x)
+{
+    if (S < 0 || H < 1 || K < 1) return ORACLE_EINVAL;
+    if (dtype != ORACLE_DTYPE_F32 && dtype != ORACLE_DTYPE_BF16) return ORACLE_EINVAL;
+    int f32 = dtype == ORACLE_DTYPE_F32;
+    for (int t = 0; t < S; ++t) {
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int32_t s = slot_of[(size_t)t * K + k];
+                if (s < 0 || (int64_t)s >= cap) continue;
+                size_t i = (size_t)s * H + h;
+                acc += f32 ? ((const float *)grad_xd)[i] : bf16_to_f32(((const uint16_t *)grad_xd)[i]);
+            }
+            size_t o = (size_t)t * H + h;
+            if (f32) ((float *)grad_x)[o] = acc;
+            else ((uint16_t *)grad_x)[o] = oracle_bf16_round(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Backward of oracle_route_topk through the gating softmax.  The weights are
+ * the softmax of the K selected logits, so for the selected experts
+ *     grad_logits[t, e_k] = w_k * (gw_k - sum_j w_j gw_j)
+ * and 0 for every expert not selected (the selection itself is piecewise
+ * constant).  fp64, rounded once to fp32.
+ */
+int oracle_route_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w, int S,
+                          int E, int K, float *grad_logits)
+{
+    if (S < 0 || E < 1 || K < 1 || K > E) return ORACLE_EINVAL;
+    for (int t = 0; t < S; ++t) {
+        double dotw = 0.0;
+        for (int k = 0; k < K; ++k)
+            dotw += (double)topk_w[(size_t)t * K + k] * (double)grad_w[(size_t)t * K + k];
+        for (int e = 0; e < E; ++e) grad_logits[(size_t)t * E + e] = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            int32_t e = topk_idx[(size_t)t * K + k];
+            if (e < 0 || e >= E) return ORACLE_EINDEX;
+            double w = topk_w[(size_t)t * K + k];
+            grad_logits[(size_t)t * E + e] = (float)(w * ((double)grad_w[(size_t)t * K + k] - dotw));
+        }
+    }
+    return ORACLE_OK;
 }
