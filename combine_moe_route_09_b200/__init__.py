@@ -26,8 +26,11 @@ from .binding import (  # noqa: F401
     lib,
     moe_capacity,
     moe_combine_dual_residual,
+    moe_combine_dual_residual_backward,
     moe_dispatch,
+    moe_dispatch_backward,
     moe_dispatch_layout,
     moe_dispatch_layout_workspace,
     moe_route_topk,
+    moe_route_topk_backward,
 )

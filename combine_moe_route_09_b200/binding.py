@@ -34,6 +34,9 @@ SIGNATURES = {
     "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
     "moe_combine_dual_residual": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_static": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _P]),
+    "moe_combine_dual_residual_backward": (_I, [_P, _P, _P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch_backward": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P]),
+    "moe_route_topk_backward": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_error_string": (ctypes.c_char_p, [_I]),
     "moe_capacity": (_L, [_I, _I, _I, _I]),
 }
@@ -243,3 +246,75 @@ def moe_combine_dual_residual(y: torch.Tensor, slot_of: torch.Tensor, topk_w: to
         _ptr(residual), _ptr(residual_out), _ptr(residual_no_routed_out), _ptr(status),
         _stream(stream, y.device)))
     return residual_out, residual_no_routed_out
+
+
+# ----------------------------------------------------------------------------------------------
+# backward (training): the transposes of the forward steps, through the same layout
+# ----------------------------------------------------------------------------------------------
+
+def moe_combine_dual_residual_backward(grad_out: torch.Tensor, y: torch.Tensor, slot_of: torch.Tensor,
+                                       topk_w: torch.Tensor, grad_no_routed=None, grad_y=None,
+                                       grad_w=None, grad_skip=None, want_skip: bool = True,
+                                       status=None, stream=None):
+    """Returns (grad_y [cap,H], grad_w [S,K] fp32, grad_skip [S,H] or None).
+
+    grad_skip is the gradient of both ``residual`` and ``shared_out``.  grad_y
+    rows that no pair maps to are not written (allocated with zeros here)."""
+    _dev(y, "y", _ACT)
+    cap, H = y.shape
+    S, K = slot_of.shape
+    _dev(grad_out, "grad_out", (y.dtype,), (S, H))
+    _dev(slot_of, "slot_of", (torch.int32,))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    if grad_no_routed is not None:
+        _dev(grad_no_routed, "grad_no_routed", (y.dtype,), (S, H))
+    if grad_y is None:
+        grad_y = torch.zeros((cap, H), dtype=y.dtype, device=y.device)
+    if grad_w is None:
+        grad_w = torch.empty((S, K), dtype=torch.float32, device=y.device)
+    if grad_skip is None and want_skip:
+        grad_skip = torch.empty((S, H), dtype=y.dtype, device=y.device)
+    _dev(grad_y, "grad_y", (y.dtype,), (cap, H))
+    _dev(grad_w, "grad_w", (torch.float32,), (S, K))
+    if grad_skip is not None:
+        _dev(grad_skip, "grad_skip", (y.dtype,), (S, H))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_combine_dual_residual_backward", lib().moe_combine_dual_residual_backward(
+        _ptr(grad_out), _ptr(grad_no_routed), _ptr(y), _dtype_code(y), S, H, K, cap, _ptr(slot_of),
+        _ptr(topk_w), _ptr(grad_y), _ptr(grad_w), _ptr(grad_skip), _ptr(status), _stream(stream, y.device)))
+    return grad_y, grad_w, grad_skip
+
+
+def moe_dispatch_backward(grad_xd: torch.Tensor, slot_of: torch.Tensor, grad_x=None, status=None,
+                          stream=None):
+    """grad_x [S,H] = sum of the K copies' gradients (straight through for FP8)."""
+    _dev(grad_xd, "grad_xd", _ACT)
+    cap, H = grad_xd.shape
+    S, K = slot_of.shape
+    _dev(slot_of, "slot_of", (torch.int32,))
+    if grad_x is None:
+        grad_x = torch.empty((S, H), dtype=grad_xd.dtype, device=grad_xd.device)
+    _dev(grad_x, "grad_x", (grad_xd.dtype,), (S, H))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_dispatch_backward", lib().moe_dispatch_backward(
+        _ptr(grad_xd), _dtype_code(grad_xd), S, H, K, cap, _ptr(slot_of), _ptr(grad_x), _ptr(status),
+        _stream(stream, grad_xd.device)))
+    return grad_x
+
+
+def moe_route_topk_backward(topk_idx: torch.Tensor, topk_w: torch.Tensor, grad_w: torch.Tensor, E: int,
+                            grad_logits=None, stream=None):
+    """grad_logits [S,E] fp32 through the gating softmax over the selected logits."""
+    _dev(topk_idx, "topk_idx", (torch.int32,))
+    S, K = topk_idx.shape
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    _dev(grad_w, "grad_w", (torch.float32,), (S, K))
+    if grad_logits is None:
+        grad_logits = torch.empty((S, E), dtype=torch.float32, device=topk_idx.device)
+    _dev(grad_logits, "grad_logits", (torch.float32,), (S, E))
+    _check("moe_route_topk_backward", lib().moe_route_topk_backward(
+        _ptr(topk_idx), _ptr(topk_w), _ptr(grad_w), S, E, K, _ptr(grad_logits),
+        _stream(stream, topk_idx.device)))
+    return grad_logits

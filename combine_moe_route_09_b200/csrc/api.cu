@@ -127,4 +127,50 @@ int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int
                                      static_cast<cudaStream_t>(stream)));
 }
 
+int moe_combine_dual_residual_backward(const void *grad_out, const void *grad_no_routed, const void *y,
+                                       int dtype, int S, int H, int K, int64_t cap, const int32_t *slot_of,
+                                       const float *topk_w, void *grad_y, float *grad_w, void *grad_skip,
+                                       int32_t *status, void *stream) {
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!slot_of || !topk_w || !grad_w || !aligned(slot_of, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (status && !aligned(status, 4)) return MOE_ERR_INVALID_ARG;
+    if (!rows_ok(grad_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if (cap > 0 && (!rows_ok(y, H, b) || !rows_ok(grad_y, H, b))) return MOE_ERR_INVALID_ARG;
+    if (grad_no_routed && !rows_ok(grad_no_routed, H, b)) return MOE_ERR_INVALID_ARG;
+    if (grad_skip && !rows_ok(grad_skip, H, b)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_combine_backward(grad_out, grad_no_routed, y, dtype, S, H, K, cap, slot_of, topk_w,
+                                              grad_y, grad_w, grad_skip, status, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_dispatch_backward(const void *grad_xd, int dtype, int S, int H, int K, int64_t cap,
+                          const int32_t *slot_of, void *grad_x, int32_t *status, void *stream) {
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!slot_of || !aligned(slot_of, 4) || (status && !aligned(status, 4))) return MOE_ERR_INVALID_ARG;
+    if ((cap > 0 && !rows_ok(grad_xd, H, b)) || !rows_ok(grad_x, H, b)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    // the combine with unit weights and no epilogue: grad_x[t] = sum_k grad_xd[slot]
+    return to_rc(moe::launch_combine(grad_xd, dtype, S, H, K, cap, slot_of, nullptr, nullptr, nullptr, grad_x,
+                                     nullptr, status, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route_topk_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w, int S, int E,
+                            int K, float *grad_logits, void *stream) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > E || K > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!topk_idx || !topk_w || !grad_w || !grad_logits) return MOE_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4) || !aligned(grad_logits, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_route_backward(topk_idx, topk_w, grad_w, S, E, K, grad_logits,
+                                            static_cast<cudaStream_t>(stream), current_sms()));
+}
+
 }  // extern "C"

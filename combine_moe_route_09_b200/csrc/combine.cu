@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
         if (first < last && lane < K) {
             const size_t o = (size_t)(first / a.nchunks) * K + lane;
             nxt = __ldg(a.slot_of + o);
-            nxt_w = __ldg(a.topk_w + o);
+            nxt_w = a.topk_w ? __ldg(a.topk_w + o) : 1.0f;  // no weights: plain sum (dispatch backward)
         }
         int i = 0;
         bool ok = true;
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
                 const int tn = t + 1;
                 if (lane < K && (long long)tn * a.nchunks < last) {
                     nxt = __ldg(a.slot_of + (size_t)tn * K + lane);
-                    nxt_w = __ldg(a.topk_w + (size_t)tn * K + lane);
+                    nxt_w = a.topk_w ? __ldg(a.topk_w + (size_t)tn * K + lane) : 1.0f;
                 }
             }
             if (i >= CB_STAGES)

@@ -101,4 +101,48 @@ cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t 
     return launch_route<32>(logits, S, E, K, idx, w, st, sms);
 }
 
+// Backward through the gating softmax: for the selected experts
+// grad_logits[t, e_k] = w_k (gw_k - sum_j w_j gw_j), 0 for the others.  One warp
+// per token: the dense row is zeroed, then lanes k < K write their entries
+// (ids outside [0, E) are skipped).
+__global__ void __launch_bounds__(256) route_backward_kernel(const int32_t *__restrict__ topk_idx,
+                                                             const float *__restrict__ topk_w,
+                                                             const float *__restrict__ grad_w, int S, int E,
+                                                             int K, float *__restrict__ grad_logits) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
+        float w = 0.f, gw = 0.f;
+        int e = -1;
+        if (lane < K) {
+            w = __ldg(topk_w + (size_t)t * K + lane);
+            gw = __ldg(grad_w + (size_t)t * K + lane);
+            e = __ldg(topk_idx + (size_t)t * K + lane);
+        }
+        float dot = __fmul_rn(w, gw);
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(FULL, dot, m);
+        float *row = grad_logits + (size_t)t * E;
+        for (int j = lane; j < E; j += 32) row[j] = 0.f;
+        __syncwarp();
+        if (lane < K && e >= 0 && e < E) row[e] = __fmul_rn(w, __fsub_rn(gw, dot));
+    }
+}
+
+cudaError_t launch_route_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w, int S,
+                                  int E, int K, float *grad_logits, cudaStream_t st, int sms) {
+    const int threads = 256;
+    int blocks = (S + 7) / 8;
+    if (blocks > sms * 8) blocks = sms * 8;
+    if (blocks < 1) blocks = 1;
+    static KernelSlots<decltype(&route_backward_kernel)> slots;
+    int n_sms = 0, per_sm = 0;
+    const cudaError_t e = slots.prepare(&route_backward_kernel, threads, 0, &n_sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(route_backward_kernel, dim3(blocks), dim3(threads), 0, st, topk_idx, topk_w, grad_w, S, E,
+                      K, grad_logits);
+}
+
 }  // namespace moe

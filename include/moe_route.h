@@ -209,6 +209,53 @@ MOE_API int moe_combine_dual_residual(const void *y, int dtype, int S, int H, in
                               const void *residual, void *residual_out,
                               void *residual_no_routed_out, int32_t *status, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* Backward of the path (training).  "MoonEP developer guide", core API      */
+/* example: the backward pass reuses the forward plan -- the gradient of the  */
+/* combine is dispatched through it and the gradient of the dispatch is       */
+/* combined back.  The same layout (slot_of) and weights are passed in.       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Backward of moe_combine_dual_residual.  With g = dL/d(residual_out) and
+ * gn = dL/d(residual_no_routed_out) (NULL: zero), per token t and pair k with
+ * 0 <= slot < cap:
+ *   grad_y    [cap, H] dtype  grad_y[slot] = w[t,k] * g[t]   (fp32 product, rounded
+ *                             once; rows no pair maps to are not written)
+ *   grad_w    [S, K] fp32     <y[slot], g[t]>  (fp32 accumulation in a fixed order;
+ *                             0 for skipped pairs)
+ *   grad_skip [S, H] dtype or NULL  g + gn: the gradient of both `residual` and
+ *                             `shared_out` (the forward adds each once to each stream)
+ * Layout, alignment and host checks as for the forward call; y is read.
+ * Device status: MOE_STATUS_BAD_SLOT for a slot >= cap (skipped), MOE_STATUS_TIMEOUT.
+ */
+MOE_API int moe_combine_dual_residual_backward(const void *grad_out, const void *grad_no_routed,
+                                               const void *y, int dtype, int S, int H, int K,
+                                               int64_t cap, const int32_t *slot_of,
+                                               const float *topk_w, void *grad_y, float *grad_w,
+                                               void *grad_skip, int32_t *status, void *stream);
+
+/*
+ * Backward of moe_dispatch: every copy of token t carried x[t], so
+ *   grad_x[t] = sum over k with 0 <= slot < cap of grad_xd[slot]   (fp32, ascending k,
+ *               rounded once; zero when no copy is valid)
+ * For the FP8 dispatch the quantiser is passed straight through: grad_xd holds
+ * the gradients of the dequantised rows, in the activation dtype.
+ *   grad_xd [cap, H] dtype (read), grad_x [S, H] dtype (written).
+ */
+MOE_API int moe_dispatch_backward(const void *grad_xd, int dtype, int S, int H, int K, int64_t cap,
+                                  const int32_t *slot_of, void *grad_x, int32_t *status, void *stream);
+
+/*
+ * Backward of moe_route_topk through the gating softmax:
+ *   grad_logits [S, E] fp32 (written, dense): w_k * (gw_k - sum_j w_j gw_j) at the
+ *   selected expert e_k, 0 elsewhere (the selection is piecewise constant).
+ * topk_idx, topk_w as produced by moe_route_topk; grad_w [S, K] fp32 = dL/dw.
+ * Ids outside [0, E) are skipped.  Host checks as for moe_route_topk.
+ */
+MOE_API int moe_route_topk_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w,
+                                    int S, int E, int K, float *grad_logits, void *stream);
+
 /*
  * moe_dispatch_layout_static: the same layout as moe_dispatch_layout, for a
  * caller that cannot allocate device memory where it makes this call -- e.g. a
