@@ -417,6 +417,119 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def backward_bytes(w) -> dict:
+    """Bytes the backward calls must move at least (padding rows excluded)."""
+    b = w.esize
+    S, H, E, K = w.S, w.H, w.E, w.K
+    gn = S * H * b if w.fused else 0
+    combine_bwd = S * H * b + gn + 2 * S * K * H * b + S * K * 12 + (S * H * b if w.fused else 0)
+    dispatch_bwd = S * K * H * b + S * H * b + S * K * 4
+    route_bwd = S * K * 12 + S * E * 4
+    return dict(combine_backward=combine_bwd, dispatch_backward=dispatch_bwd, route_backward=route_bwd)
+
+
+def run_backward(args, w, rank, world, local_rank):
+    """Times the training backward of the pass: combine backward (grad_y, grad_w and,
+    with the dual residual, the skip gradient), dispatch backward of a synthetic
+    expert-input gradient, and the router backward; forward state from one forward pass."""
+    import numpy as np
+    import torch
+
+    from combine_moe_route_09_b200 import binding as B
+    from combine_moe_route_09_b200 import synth
+    from combine_moe_route_09_b200.buffer import MoeBuffer
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    inp = host_inputs(w)
+    d = {k: synth.to_torch(v, device=device) for k, v in inp.items()}
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device)
+    sh, rs = (d["shared"], d["residual"]) if w.fused else (None, None)
+    buf.step(d["logits"], d["x"], d["y"], sh, rs)
+    torch.cuda.synchronize()
+    gen = torch.Generator(device=device).manual_seed(w.seed + 1000)
+    g = torch.randn((w.S, w.H), generator=gen, device=device).to(dt)
+    gn = torch.randn((w.S, w.H), generator=gen, device=device).to(dt) if w.fused else None
+    gxd = torch.randn((buf.cap, w.H), generator=gen, device=device).to(dt)
+    grad_y = torch.zeros((buf.cap, w.H), dtype=dt, device=device)
+    grad_w = torch.empty((w.S, w.K), dtype=torch.float32, device=device)
+    skip = torch.empty((w.S, w.H), dtype=dt, device=device) if w.fused else None
+    grad_x = torch.empty((w.S, w.H), dtype=dt, device=device)
+    grad_logits = torch.empty((w.S, w.E), dtype=torch.float32, device=device)
+    status = buf.status
+    slot = buf.layout.slot_of
+
+    calls = [
+        ("combine_backward", lambda: B.moe_combine_dual_residual_backward(
+            g, d["y"], slot, buf.topk_w, grad_no_routed=gn, grad_y=grad_y, grad_w=grad_w, grad_skip=skip,
+            want_skip=w.fused, status=status)),
+        ("dispatch_backward", lambda: B.moe_dispatch_backward(gxd, slot, grad_x=grad_x, status=status)),
+        ("route_backward", lambda: B.moe_route_topk_backward(buf.topk_idx, buf.topk_w, grad_w, w.E,
+                                                             grad_logits=grad_logits)),
+    ]
+
+    def eager():
+        for _, f in calls:
+            f()
+
+    for _ in range(args.warmup):
+        eager()
+    torch.cuda.synchronize()
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            eager()
+        graph.replay()
+        torch.cuda.synchronize()
+    if buf.read_status() != 0:
+        raise RuntimeError("device status flagged a problem")
+    K = args.steps
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(K):
+        graph.replay() if graph is not None else eager()
+    b.record()
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(a.elapsed_time(b), world, device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record()
+        for j, (_, f) in enumerate(calls):
+            f()
+            ev[i][j + 1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if buf.read_status() != 0:
+        raise RuntimeError("device status flagged a problem")
+    if rank != 0:
+        return
+    ab = backward_bytes(w)
+    peak, peak_kind = read_peak_hbm()
+    phases = {}
+    for j, (name, _) in enumerate(calls):
+        ms = statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
+        gbs = ab[name] / (ms * 1e-3) / 1e9
+        phases[name] = {"us": ms * 1e3, "algorithmic_bytes": ab[name], "gb_s": gbs, "frac_of_peak": gbs / peak}
+    cb = phases["combine_backward"]
+    line = {
+        "mode": "backward", "metric": "backward pass tokens/s (combine, dispatch and router backward), 1 GPU",
+        "value": w.S * world * K / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": workload_config(w, world), "phases": phases,
+        "roofline": {"kernel": "combine_bwd_kernel", "bound": "hbm", "achieved": cb["gb_s"], "peak": peak,
+                     "unit": "GB/s", "frac": cb["gb_s"] / peak, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": ab["combine_backward"], "traffic": None},
+        "gpu_launches": K * 3, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,6 +543,8 @@ def main(argv=None):
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time the value pass as CUDA-graph replays of one step (default; "
                          "--no-graph times eager calls)")
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward"],
+                    help="forward: the routing pass (default); backward: its training backward")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override S (a smaller case of the same workload, for profiling)")
     args = ap.parse_args(argv)
@@ -456,7 +571,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if args.mode == "backward":
+            run_backward(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
