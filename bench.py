@@ -530,6 +530,63 @@ def run_backward(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8_combine(args, w, rank, world, local_rank):
+    """Times the combine over FP8 expert outputs (e4m3 + 128-channel scales) on the
+    workload's shapes; the expert outputs are a seeded N(0,1) buffer quantised
+    once by the FP8 dispatch kernel (identity slots)."""
+    import torch
+
+    from combine_moe_route_09_b200 import binding as B
+    from combine_moe_route_09_b200 import synth
+    from combine_moe_route_09_b200.buffer import MoeBuffer
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    inp = host_inputs(w)
+    d = {k: synth.to_torch(v, device=device) for k, v in inp.items()}
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device)
+    sh, rs = (d["shared"], d["residual"]) if w.fused else (None, None)
+    buf.step(d["logits"], d["x"], d["y"], sh, rs)
+    ident = torch.arange(buf.cap, dtype=torch.int32, device=device).reshape(-1, 1)
+    yq, ys = B.moe_dispatch(d["y"], ident, buf.cap, B.MOE_QUANT_FP8_E4M3_B128)
+    out = torch.empty((w.S, w.H), dtype=dt, device=device)
+    rnr = torch.empty((w.S, w.H), dtype=dt, device=device) if w.fused else None
+
+    def call():
+        B.moe_combine_fp8_dual_residual(yq, ys, buf.layout.slot_of, buf.topk_w, shared_out=sh, residual=rs,
+                                        residual_out=out, residual_no_routed_out=rnr, want_no_routed=w.fused,
+                                        dtype=dt, status=buf.status)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ev[0].record()
+    for i in range(K):
+        call()
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if buf.read_status() != 0:
+        raise RuntimeError("device status flagged a problem")
+    if rank != 0:
+        return
+    ms = statistics.fmean(ev[i].elapsed_time(ev[i + 1]) for i in range(K))
+    S, H, Kk, b = w.S, w.H, w.K, w.esize
+    nbytes = S * Kk * H + S * Kk * (H // 128) * 4 + S * Kk * 8 + (4 * S * H * b if w.fused else S * H * b)
+    peak, peak_kind = read_peak_hbm()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"mode": "fp8_combine", "metric": "combine over FP8 expert outputs, tokens/s, 1 GPU",
+                      "value": S / (ms * 1e-3), "unit": "tokens/s", "us_per_call": ms * 1e3,
+                      "algorithmic_bytes": nbytes, "gb_s": gbs, "frac_of_peak": gbs / peak,
+                      "peak_source": peak_kind, "config": workload_config(w, world), "clocks": clocks,
+                      "steps": K, "warmup": args.warmup}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,8 +600,9 @@ def main(argv=None):
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time the value pass as CUDA-graph replays of one step (default; "
                          "--no-graph times eager calls)")
-    ap.add_argument("--mode", default="forward", choices=["forward", "backward"],
-                    help="forward: the routing pass (default); backward: its training backward")
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward", "fp8_combine"],
+                    help="forward: the routing pass (default); backward: its training backward; "
+                         "fp8_combine: the combine over FP8 expert outputs")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override S (a smaller case of the same workload, for profiling)")
     args = ap.parse_args(argv)
@@ -573,6 +631,8 @@ def main(argv=None):
     try:
         if args.mode == "backward":
             run_backward(args, w, rank, world, local_rank)
+        elif args.mode == "fp8_combine":
+            run_fp8_combine(args, w, rank, world, local_rank)
         else:
             run_ours(args, w, rank, world, local_rank)
     finally:

@@ -27,6 +27,7 @@ from .binding import (  # noqa: F401
     moe_capacity,
     moe_combine_dual_residual,
     moe_combine_dual_residual_backward,
+    moe_combine_fp8_dual_residual,
     moe_dispatch,
     moe_dispatch_backward,
     moe_dispatch_layout,

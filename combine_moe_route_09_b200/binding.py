@@ -34,6 +34,7 @@ SIGNATURES = {
     "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
     "moe_combine_dual_residual": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_static": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _P]),
+    "moe_combine_fp8_dual_residual": (_I, [_P, _P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine_dual_residual_backward": (_I, [_P, _P, _P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_backward": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P]),
     "moe_route_topk_backward": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
@@ -245,6 +246,37 @@ def moe_combine_dual_residual(y: torch.Tensor, slot_of: torch.Tensor, topk_w: to
         _ptr(y), _dtype_code(y), S, H, K, cap, _ptr(slot_of), _ptr(topk_w), _ptr(shared_out),
         _ptr(residual), _ptr(residual_out), _ptr(residual_no_routed_out), _ptr(status),
         _stream(stream, y.device)))
+    return residual_out, residual_no_routed_out
+
+
+def moe_combine_fp8_dual_residual(yq: torch.Tensor, ys: torch.Tensor, slot_of: torch.Tensor,
+                                  topk_w: torch.Tensor, shared_out=None, residual=None, residual_out=None,
+                                  residual_no_routed_out=None, want_no_routed: bool = True,
+                                  dtype: torch.dtype = torch.bfloat16, status=None, stream=None):
+    """moe_combine_dual_residual over FP8 expert outputs: yq [cap,H] e4m3 codes and
+    ys [cap,H/128] fp32 block scales; outputs (and shared_out/residual) in ``dtype``."""
+    _dev(yq, "yq", _FP8)
+    cap, H = yq.shape
+    S, K = slot_of.shape
+    _dev(ys, "ys", (torch.float32,), (cap, H // 128))
+    _dev(slot_of, "slot_of", (torch.int32,))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    for name, t in (("shared_out", shared_out), ("residual", residual)):
+        if t is not None:
+            _dev(t, name, (dtype,), (S, H))
+    if residual_out is None:
+        residual_out = torch.empty((S, H), dtype=dtype, device=yq.device)
+    _dev(residual_out, "residual_out", (dtype,), (S, H))
+    if residual_no_routed_out is None and want_no_routed and shared_out is not None and residual is not None:
+        residual_no_routed_out = torch.empty((S, H), dtype=dtype, device=yq.device)
+    if residual_no_routed_out is not None:
+        _dev(residual_no_routed_out, "residual_no_routed_out", (dtype,), (S, H))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    code = MOE_DTYPE_F32 if dtype == torch.float32 else MOE_DTYPE_BF16
+    _check("moe_combine_fp8_dual_residual", lib().moe_combine_fp8_dual_residual(
+        _ptr(yq), _ptr(ys), code, S, H, K, cap, _ptr(slot_of), _ptr(topk_w), _ptr(shared_out), _ptr(residual),
+        _ptr(residual_out), _ptr(residual_no_routed_out), _ptr(status), _stream(stream, yq.device)))
     return residual_out, residual_no_routed_out
 
 

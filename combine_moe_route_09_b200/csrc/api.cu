@@ -127,6 +127,29 @@ int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int
                                      static_cast<cudaStream_t>(stream)));
 }
 
+int moe_combine_fp8_dual_residual(const uint8_t *yq, const float *ys, int dtype, int S, int H, int K, int64_t cap,
+                                  const int32_t *slot_of, const float *topk_w, const void *shared_out,
+                                  const void *residual, void *residual_out, void *residual_no_routed_out,
+                                  int32_t *status, void *stream) {
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || H % 512 != 0 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 ||
+        cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (residual_no_routed_out && !(shared_out && residual)) return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!slot_of || !topk_w || !aligned(slot_of, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+    if (status && !aligned(status, 4)) return MOE_ERR_INVALID_ARG;
+    if (cap > 0 && (!rows_ok(yq, H, 1) || !ys || !aligned(ys, 16))) return MOE_ERR_INVALID_ARG;
+    if (!rows_ok(residual_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if (shared_out && !rows_ok(shared_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if (residual && !rows_ok(residual, H, b)) return MOE_ERR_INVALID_ARG;
+    if (residual_no_routed_out && !rows_ok(residual_no_routed_out, H, b)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_combine_fp8(yq, ys, dtype, S, H, K, cap, slot_of, topk_w, shared_out, residual,
+                                         residual_out, residual_no_routed_out, status,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int moe_combine_dual_residual_backward(const void *grad_out, const void *grad_no_routed, const void *y,
                                        int dtype, int S, int H, int K, int64_t cap, const int32_t *slot_of,
                                        const float *topk_w, void *grad_y, float *grad_w, void *grad_skip,

@@ -42,6 +42,11 @@ cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_
                            const void *residual, void *out, void *out_no_routed, int32_t *status,
                            cudaStream_t st);
 
+cudaError_t launch_combine_fp8(const uint8_t *yq, const float *ys, int dtype, int S, int H, int K, int64_t cap,
+                               const int32_t *slot_of, const float *topk_w, const void *shared_out,
+                               const void *residual, void *out, void *out_no_routed, int32_t *status,
+                               cudaStream_t st);
+
 cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y, int dtype, int S, int H,
                                     int K, int64_t cap, const int32_t *slot_of, const float *topk_w,
                                     void *grad_y, float *grad_w, void *grad_skip, int32_t *status,

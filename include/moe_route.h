@@ -209,6 +209,23 @@ MOE_API int moe_combine_dual_residual(const void *y, int dtype, int S, int H, in
                               const void *residual, void *residual_out,
                               void *residual_no_routed_out, int32_t *status, void *stream);
 
+/*
+ * Combine over FP8 expert outputs: moe_combine_dual_residual with y given as
+ * e4m3 codes plus one fp32 scale per 128-channel block -- the format of the FP8
+ * dispatch ("Efficient and portable mixture-of-experts communication",
+ * Dispatch: tokens travel with their block scaling factors).  Each gathered
+ * element is dequantised as y = e4m3_value(q) * scale (an fp32 product); the
+ * accumulation (fp32, ascending k) and the epilogue are those of
+ * moe_combine_dual_residual, whose shared_out / residual / outputs here have
+ * type `dtype`.
+ *   yq [cap, H] uint8 e4m3 (16-byte aligned), ys [cap, H/128] fp32 (16-byte aligned)
+ * Host checks as for moe_combine_dual_residual, plus H % 512 == 0.
+ */
+MOE_API int moe_combine_fp8_dual_residual(const uint8_t *yq, const float *ys, int dtype, int S, int H, int K,
+                                          int64_t cap, const int32_t *slot_of, const float *topk_w,
+                                          const void *shared_out, const void *residual, void *residual_out,
+                                          void *residual_no_routed_out, int32_t *status, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Backward of the path (training).  "MoonEP developer guide", core API      */
 /* example: the backward pass reuses the forward plan -- the gradient of the  */

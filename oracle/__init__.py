@@ -51,6 +51,7 @@ def _load():
         lib.oracle_layout.argtypes = [P, I, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch.argtypes = [P, I, I, I, I, P, I, L, P, P]
         lib.oracle_combine.argtypes = [P, I, I, I, I, L, P, P, P, P, P, P]
+        lib.oracle_combine_fp8.argtypes = [P, P, I, I, I, I, L, P, P, P, P, P, P]
         lib.oracle_combine_backward.argtypes = [P, P, P, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch_backward.argtypes = [P, I, I, I, I, L, P, P]
         lib.oracle_route_backward.argtypes = [P, P, P, I, I, I, P]
@@ -170,6 +171,30 @@ def combine(y: np.ndarray, slot_of: np.ndarray, topk_w: np.ndarray, shared=None,
                                 _ptr(shared), _ptr(residual), _ptr(out), _ptr(rnr))
     if rc:
         raise OracleError("oracle_combine", rc)
+    return out, rnr
+
+
+def combine_fp8(yq, ys, slot_of, topk_w, shared=None, residual=None, dtype="bf16",
+                want_no_routed: bool = True):
+    """Combine over e4m3 expert outputs yq [cap,H] (uint8) with scales ys [cap,H/128].
+
+    The outputs (and shared/residual, if given) are in ``dtype`` ("bf16" or "f32")."""
+    yq = _c(yq, np.uint8)
+    ys = _c(ys, np.float32)
+    slot_of = _c(slot_of, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    S, K = slot_of.shape
+    cap, H = yq.shape
+    code = DTYPE_BF16 if dtype == "bf16" else DTYPE_F32
+    npdt = np.uint16 if dtype == "bf16" else np.float32
+    shared = None if shared is None else _c(shared, npdt)
+    residual = None if residual is None else _c(residual, npdt)
+    out = np.empty((S, H), npdt)
+    rnr = np.empty((S, H), npdt) if (want_no_routed and shared is not None and residual is not None) else None
+    rc = _load().oracle_combine_fp8(_ptr(yq), _ptr(ys), code, S, H, K, cap, _ptr(slot_of), _ptr(topk_w),
+                                    _ptr(shared), _ptr(residual), _ptr(out), _ptr(rnr))
+    if rc:
+        raise OracleError("oracle_combine_fp8", rc)
     return out, rnr
 
 

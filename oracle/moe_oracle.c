@@ -13,6 +13,7 @@
  *   oracle_layout       per-expert counts, padded offsets, slot assignment
  *   oracle_dispatch     scatter of token rows (optionally FP8 e4m3, 128-ch blocks)
  *   oracle_combine      gather + top-K weighted sum + dual-residual epilogue
+ *   oracle_combine_fp8  the combine over e4m3 expert outputs with block scales
  *   oracle_combine_backward / oracle_dispatch_backward / oracle_route_backward
  *                       the transposes of the steps (training)
  *   oracle_e4m3_encode / oracle_e4m3_decode / oracle_bf16_round   format helpers
@@ -490,4 +491,56 @@ int oracle_route_backward(const int32_t *topk_idx, const float *topk_w, const fl
         }
     }
     return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Combine over FP8 expert outputs                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * oracle_combine with the expert outputs given as e4m3 codes plus one fp32
+ * scale per 128-channel block (the format of the FP8 dispatch; "Efficient and
+ * portable mixture-of-experts communication", Dispatch: tokens travel with
+ * their block scaling factors).  Each element is dequantised as
+ *     y = e4m3_value(q[slot, h]) * s[slot, h / 128]     (fp32 product)
+ * and the accumulation and epilogue are those of oracle_combine; the
+ * remaining arrays are in `dtype`.  H % 128 == 0.
+ */
+int oracle_combine_fp8(const uint8_t *yq, const float *ys, int dtype, int S, int H, int K, int64_t cap,
+                       const int32_t *slot_of, const float *topk_w, const void *shared,
+                       const void *residual, void *out, void *out_no_routed)
+{
+    if (S < 0 || H < 1 || K < 1 || H % 128 != 0) return ORACLE_EINVAL;
+    if (dtype != ORACLE_DTYPE_F32 && dtype != ORACLE_DTYPE_BF16) return ORACLE_EINVAL;
+    if (out_no_routed && !(shared && residual)) return ORACLE_EINVAL;
+    int nb = H / 128, f32 = dtype == ORACLE_DTYPE_F32, rc = ORACLE_OK;
+    for (int t = 0; t < S; ++t) {
+        for (int k = 0; k < K; ++k) {
+            int32_t s = slot_of[(size_t)t * K + k];
+            if (s >= 0 && (int64_t)s >= cap) rc = ORACLE_EOVERFLOW;
+        }
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int32_t s = slot_of[(size_t)t * K + k];
+                if (s < 0 || (int64_t)s >= cap) continue;
+                float yv = oracle_e4m3_decode(yq[(size_t)s * H + h]) * ys[(size_t)s * nb + h / 128];
+                acc = fmaf(topk_w[(size_t)t * K + k], yv, acc);
+            }
+            size_t oi = (size_t)t * H + h;
+            float sh = 0.0f, rs = 0.0f;
+            if (shared) sh = f32 ? ((const float *)shared)[oi] : bf16_to_f32(((const uint16_t *)shared)[oi]);
+            if (residual) rs = f32 ? ((const float *)residual)[oi] : bf16_to_f32(((const uint16_t *)residual)[oi]);
+            float m = shared ? sh + acc : acc;
+            float o = residual ? rs + m : m;
+            if (f32) ((float *)out)[oi] = o;
+            else ((uint16_t *)out)[oi] = oracle_bf16_round(o);
+            if (out_no_routed) {
+                float n = rs + sh;
+                if (f32) ((float *)out_no_routed)[oi] = n;
+                else ((uint16_t *)out_no_routed)[oi] = oracle_bf16_round(n);
+            }
+        }
+    }
+    return rc;
 }

@@ -113,3 +113,30 @@ def test_combine_k_order_is_fixed(oracle_lib):
     assert out[0, 0] == 0.0
     out2, _ = oracle_lib.combine(y, np.array([[0, 2, 1]], np.int32), np.ones((1, 3), np.float32))
     assert out2[0, 0] == 1.0
+
+
+@pytest.mark.parametrize("name,S", [("4", 48), ("3", 32)])
+def test_combine_fp8_equals_combine_of_dequantised_rows(oracle_lib, name, S):
+    """The FP8-input combine equals the fp32 combine of rows dequantised independently:
+    torch's e4m3 decode, times the block scale in numpy fp32."""
+    import torch
+
+    w = synth.WORKLOADS[name].replace(S=S)
+    x = synth.activations(w)
+    idx, wt, lay = _route_layout(oracle_lib, w)
+    yq, ys = oracle_lib.dispatch(x, lay["slot_of"], lay["cap"], quant=oracle_lib.QUANT_FP8_E4M3_B128)
+    deq = torch.from_numpy(yq).view(torch.float8_e4m3fn).float().numpy()
+    deq = (deq * np.repeat(ys, 128, axis=1)).astype(np.float32)          # fp32 product
+    rng = np.random.default_rng(5)
+    sh = rng.standard_normal((S, w.H)).astype(np.float32)
+    rs = rng.standard_normal((S, w.H)).astype(np.float32)
+    for kw in (dict(), dict(shared=sh, residual=rs)):
+        ref, ref_n = oracle_lib.combine(deq, lay["slot_of"], wt, **kw)
+        got, got_n = oracle_lib.combine_fp8(yq, ys, lay["slot_of"], wt, dtype="f32", **kw)
+        np.testing.assert_array_equal(got, ref)
+        if kw:
+            np.testing.assert_array_equal(got_n, ref_n)
+    # identity round trip through the quantiser: within the e4m3 error bound
+    out, _ = oracle_lib.combine_fp8(yq, ys, lay["slot_of"], wt, dtype="f32")
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    assert np.all(np.abs(out - xf) <= 2.0 ** -4 * np.abs(xf) + np.repeat(ys[lay["slot_of"][:, 0]], 128, 1) * 2.0 ** -9)
