@@ -51,6 +51,11 @@ def _load():
         lib.oracle_layout.argtypes = [P, I, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch.argtypes = [P, I, I, I, I, P, I, L, P, P]
         lib.oracle_combine.argtypes = [P, I, I, I, I, L, P, P, P, P, P, P]
+        lib.oracle_route_sigmoid_grouped.argtypes = [P, P, I, I, I, I, I, I, ctypes.c_float, P, P]
+        lib.oracle_route_exp.argtypes = [ctypes.c_float]
+        lib.oracle_route_exp.restype = ctypes.c_float
+        lib.oracle_route_sigmoid.argtypes = [ctypes.c_float]
+        lib.oracle_route_sigmoid.restype = ctypes.c_float
         lib.oracle_combine_fp8.argtypes = [P, P, I, I, I, I, L, P, P, P, P, P, P]
         lib.oracle_combine_backward.argtypes = [P, P, P, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch_backward.argtypes = [P, I, I, I, I, L, P, P]
@@ -99,6 +104,31 @@ def route_topk(logits: np.ndarray, K: int):
     if rc:
         raise OracleError("oracle_route_topk", rc)
     return idx, w
+
+
+def route_sigmoid_grouped(logits, K: int, bias=None, n_group: int = 1, topk_group: int = 1,
+                          normalize: bool = True, scale: float = 1.0):
+    """Sigmoid scores, selection-only bias, group-limited top-K; see moe_oracle.c."""
+    logits = _c(logits, np.float32)
+    S, E = logits.shape
+    bias = None if bias is None else _c(bias, np.float32)
+    idx = np.empty((S, K), np.int32)
+    w = np.empty((S, K), np.float32)
+    rc = _load().oracle_route_sigmoid_grouped(_ptr(logits), _ptr(bias), S, E, K, n_group, topk_group,
+                                              int(normalize), float(scale), _ptr(idx), _ptr(w))
+    if rc:
+        raise OracleError("oracle_route_sigmoid_grouped", rc)
+    return idx, w
+
+
+def route_exp(x: np.ndarray) -> np.ndarray:
+    f = _load().oracle_route_exp
+    return np.array([f(float(v)) for v in np.asarray(x, np.float32).ravel()], np.float32)
+
+
+def route_sigmoid(x: np.ndarray) -> np.ndarray:
+    f = _load().oracle_route_sigmoid
+    return np.array([f(float(v)) for v in np.asarray(x, np.float32).ravel()], np.float32)
 
 
 def capacity(S: int, E: int, K: int, P: int) -> int:

@@ -14,6 +14,8 @@
  *   oracle_dispatch     scatter of token rows (optionally FP8 e4m3, 128-ch blocks)
  *   oracle_combine      gather + top-K weighted sum + dual-residual epilogue
  *   oracle_combine_fp8  the combine over e4m3 expert outputs with block scales
+ *   oracle_route_sigmoid_grouped   router variant: sigmoid scores, selection-only
+ *                       bias, group-limited top-K (with its exp / sigmoid)
  *   oracle_combine_backward / oracle_dispatch_backward / oracle_route_backward
  *                       the transposes of the steps (training)
  *   oracle_e4m3_encode / oracle_e4m3_decode / oracle_bf16_round   format helpers
@@ -543,4 +545,117 @@ int oracle_combine_fp8(const uint8_t *yq, const float *ys, int dtype, int S, int
         }
     }
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router variant: sigmoid scores, selection-only bias, group-limited top-K   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * exp(x) in fp32 from IEEE basic operations only, so that this oracle and the
+ * CUDA kernel evaluate exactly the same sequence and take the same routing
+ * decisions: Cody-Waite reduction x = n ln2 + r (n = RN(x log2 e), ln 2 split
+ * into a 16-bit head, exact for |n| <= 256, and a tail), exp(r) by the degree-7
+ * Taylor polynomial in Horner form with fma (|r| <= 0.35: truncation < 3e-9
+ * relative), and 2^n applied as two exact power-of-two factors.  Pinned against
+ * fp64 exp (within 2 ulp).  Below -104 the result is 0, above 88.72 it is inf.
+ */
+static float pow2i(int e) { return bits_to_f32((uint32_t)(e + 127) << 23); } /* -126 <= e <= 127 */
+
+float oracle_route_exp(float x)
+{
+    if (x > 88.72283935546875f) return INFINITY;
+    if (x < -103.97208404541015625f) return 0.0f;
+    const float log2e = 1.44269502162933349609375f;       /* RN(1/ln 2) */
+    const float ln2_hi = 0.693145751953125f;               /* ln 2 to 16 bits */
+    const float ln2_lo = 1.428606765330187045037746429443359375e-06f; /* RN(ln 2 - ln2_hi) */
+    float n = rintf(x * log2e);
+    float r = fmaf(-n, ln2_hi, x);
+    r = fmaf(-n, ln2_lo, r);
+    float p = 1.9841270114e-04f;                /* 1/7! */
+    p = fmaf(p, r, 1.3888889225e-03f);          /* 1/6! */
+    p = fmaf(p, r, 8.3333337680e-03f);          /* 1/5! */
+    p = fmaf(p, r, 4.1666667908e-02f);          /* 1/4! */
+    p = fmaf(p, r, 1.6666667163e-01f);          /* 1/3! */
+    p = fmaf(p, r, 0.5f);                       /* 1/2! */
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ni = (int)n;
+    int h = ni / 2;
+    return (p * pow2i(h)) * pow2i(ni - h);
+}
+
+/* sigmoid(l) = 1 / (1 + exp(-l)), fp32, IEEE addition and division. */
+float oracle_route_sigmoid(float l) { return 1.0f / (1.0f + oracle_route_exp(-l)); }
+
+/*
+ * Sigmoid routing with a selection-only bias and group-limited top-K (the
+ * DeepSeek-V3 technical report, which "Efficient and portable
+ * mixture-of-experts communication" cites for its router; the pages give no
+ * detail, so this is the plainest reading):
+ *   s_e = sigmoid(l_e)                          (the gating score)
+ *   c_e = s_e + bias_e                          (the selection score; bias may be NULL)
+ *   n_group > 1: the E experts form n_group contiguous groups; a group's score
+ *     is (largest c) + (second largest c) in it (fp32, in that order); the
+ *     topk_group highest groups (ties: lower group) stay, the rest are excluded
+ *   top-K of c over the experts that stay (descending, ties: lower id)
+ *   w_k = s_{e_k}; with normalize, w_k = s_{e_k} / (s_{e_0} + ... + s_{e_{K-1}})
+ *     (sum in k order); then w_k = w_k * scale.   All fp32.
+ * Requires E % n_group == 0, E / n_group >= 2, topk_group * E / n_group >= K.
+ */
+int oracle_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                                 int topk_group, int normalize, float scale, int32_t *topk_idx, float *topk_w)
+{
+    if (S < 0 || E < 1 || K < 1 || K > E || n_group < 1 || E % n_group != 0) return ORACLE_EINVAL;
+    int gsize = E / n_group;
+    if (n_group > 1 && (gsize < 2 || topk_group < 1 || topk_group > n_group || topk_group * gsize < K))
+        return ORACLE_EINVAL;
+    float *s = (float *)malloc(sizeof(float) * (size_t)E);
+    float *c = (float *)malloc(sizeof(float) * (size_t)E);
+    char *allowed = (char *)malloc((size_t)E);
+    float *gs = (float *)malloc(sizeof(float) * (size_t)n_group);
+    char *gtaken = (char *)malloc((size_t)n_group);
+    if (!s || !c || !allowed || !gs || !gtaken) { free(s); free(c); free(allowed); free(gs); free(gtaken); return ORACLE_EINVAL; }
+    for (int t = 0; t < S; ++t) {
+        const float *row = logits + (size_t)t * E;
+        for (int e = 0; e < E; ++e) {
+            s[e] = oracle_route_sigmoid(row[e]);
+            c[e] = bias ? s[e] + bias[e] : s[e];
+            allowed[e] = 1;
+        }
+        if (n_group > 1) {
+            for (int g = 0; g < n_group; ++g) {
+                int b1 = -1, b2 = -1;
+                for (int e = g * gsize; e < (g + 1) * gsize; ++e) {
+                    if (b1 < 0 || c[e] > c[b1]) { b2 = b1; b1 = e; }
+                    else if (b2 < 0 || c[e] > c[b2]) b2 = e;
+                }
+                gs[g] = c[b1] + c[b2];
+                gtaken[g] = 0;
+            }
+            for (int r = 0; r < topk_group; ++r) {
+                int best = -1;
+                for (int g = 0; g < n_group; ++g)
+                    if (!gtaken[g] && (best < 0 || gs[g] > gs[best])) best = g;
+                gtaken[best] = 1;
+            }
+            for (int e = 0; e < E; ++e) allowed[e] = gtaken[e / gsize];
+        }
+        for (int k = 0; k < K; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (allowed[e] && (best < 0 || c[e] > c[best])) best = e;
+            allowed[best] = 0;
+            topk_idx[(size_t)t * K + k] = best;
+        }
+        float sum = 0.0f;
+        for (int k = 0; k < K; ++k) sum += s[topk_idx[(size_t)t * K + k]];
+        for (int k = 0; k < K; ++k) {
+            float v = s[topk_idx[(size_t)t * K + k]];
+            if (normalize) v = v / sum;
+            topk_w[(size_t)t * K + k] = v * scale;
+        }
+    }
+    free(s); free(c); free(allowed); free(gs); free(gtaken);
+    return ORACLE_OK;
 }
