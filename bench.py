@@ -587,6 +587,57 @@ def run_fp8_combine(args, w, rank, world, local_rank):
                       "steps": K, "warmup": args.warmup}), flush=True)
 
 
+def run_router(args, w, rank, world, local_rank):
+    """Times the two routers on the workload's logits: the softmax top-K of the
+    routing pass and the variant (sigmoid scores, selection-only bias, n_group=8
+    groups of which topk_group=4 are kept, normalised, scale 2.5)."""
+    import numpy as np
+    import torch
+
+    from combine_moe_route_09_b200 import binding as B
+    from combine_moe_route_09_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    logits = synth.to_torch(synth.logits(w), device=device)
+    bias = torch.from_numpy((np.random.default_rng(w.seed).standard_normal(w.E) * 0.05).astype(np.float32)).to(device)
+    idx = torch.empty((w.S, w.K), dtype=torch.int32, device=device)
+    wt = torch.empty((w.S, w.K), dtype=torch.float32, device=device)
+    n_group = 8 if w.E % 8 == 0 and w.E // 8 >= 2 and 4 * (w.E // 8) >= w.K else 1
+    calls = {
+        "route_topk_softmax": lambda: B.moe_route_topk(logits, w.K, topk_idx=idx, topk_w=wt),
+        "route_sigmoid_grouped": lambda: B.moe_route_sigmoid_grouped(
+            logits, w.K, bias=bias, n_group=n_group, topk_group=4 if n_group > 1 else 1, normalize=True,
+            scale=2.5, topk_idx=idx, topk_w=wt),
+    }
+    nbytes = w.S * w.E * 4 + w.S * w.K * 8 + (w.E * 4)
+    peak, peak_kind = read_peak_hbm()
+    res = {}
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    for name, call in calls.items():
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for _ in range(args.steps):
+            call()
+        ev1.record()
+        torch.cuda.synchronize()
+        us = ev0.elapsed_time(ev1) * 1e3 / args.steps
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"us_per_call": us, "tokens_per_s": w.S / (us * 1e-6), "gb_s": gbs, "frac_of_peak": gbs / peak}
+    clocks = sampler.stop()
+    if rank != 0:
+        return
+    print(json.dumps({"mode": "router", "metric": "router tokens/s, 1 GPU (back-to-back launches)",
+                      "value": res["route_sigmoid_grouped"]["tokens_per_s"], "unit": "tokens/s",
+                      "routers": res, "algorithmic_bytes": nbytes, "peak_source": peak_kind,
+                      "n_group": n_group, "config": workload_config(w, world), "clocks": clocks,
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,9 +651,9 @@ def main(argv=None):
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time the value pass as CUDA-graph replays of one step (default; "
                          "--no-graph times eager calls)")
-    ap.add_argument("--mode", default="forward", choices=["forward", "backward", "fp8_combine"],
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward", "fp8_combine", "router"],
                     help="forward: the routing pass (default); backward: its training backward; "
-                         "fp8_combine: the combine over FP8 expert outputs")
+                         "fp8_combine: the combine over FP8 expert outputs; router: both routers")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override S (a smaller case of the same workload, for profiling)")
     args = ap.parse_args(argv)
@@ -633,6 +684,8 @@ def main(argv=None):
             run_backward(args, w, rank, world, local_rank)
         elif args.mode == "fp8_combine":
             run_fp8_combine(args, w, rank, world, local_rank)
+        elif args.mode == "router":
+            run_router(args, w, rank, world, local_rank)
         else:
             run_ours(args, w, rank, world, local_rank)
     finally:

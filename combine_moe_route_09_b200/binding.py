@@ -29,6 +29,7 @@ _P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 # name -> (restype, argtypes), the exact C signatures
 SIGNATURES = {
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_route_sigmoid_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _Z, _P, _P]),
     "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
@@ -117,6 +118,26 @@ def moe_route_topk(logits: torch.Tensor, K: int, topk_idx=None, topk_w=None, str
     _dev(topk_w, "topk_w", (torch.float32,), (S, K))
     _check("moe_route_topk", lib().moe_route_topk(_ptr(logits), S, E, K, _ptr(topk_idx), _ptr(topk_w),
                                                    _stream(stream, logits.device)))
+    return topk_idx, topk_w
+
+
+def moe_route_sigmoid_grouped(logits: torch.Tensor, K: int, bias=None, n_group: int = 1,
+                              topk_group: int = 1, normalize: bool = True, scale: float = 1.0,
+                              topk_idx=None, topk_w=None, stream=None):
+    """Sigmoid scores, selection-only bias, group-limited top-K (see include/moe_route.h)."""
+    _dev(logits, "logits", (torch.float32,))
+    S, E = logits.shape
+    if bias is not None:
+        _dev(bias, "bias", (torch.float32,), (E,))
+    if topk_idx is None:
+        topk_idx = torch.empty((S, K), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((S, K), dtype=torch.float32, device=logits.device)
+    _dev(topk_idx, "topk_idx", (torch.int32,), (S, K))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    _check("moe_route_sigmoid_grouped", lib().moe_route_sigmoid_grouped(
+        _ptr(logits), _ptr(bias), S, E, K, n_group, topk_group, int(normalize), float(scale), _ptr(topk_idx),
+        _ptr(topk_w), _stream(stream, logits.device)))
     return topk_idx, topk_w
 
 

@@ -57,6 +57,24 @@ int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, 
                                         static_cast<cudaStream_t>(stream), current_sms()));
 }
 
+int moe_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                              int topk_group, int normalize, float scale, int32_t *topk_idx, float *topk_w,
+                              void *stream) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > E || K > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+    if (n_group < 1 || n_group > MOE_MAX_GROUPS || E % n_group != 0) return MOE_ERR_INVALID_ARG;
+    if (n_group > 1 && (E / n_group < 2 || topk_group < 1 || topk_group > n_group ||
+                        (int64_t)topk_group * (E / n_group) < K))
+        return MOE_ERR_INVALID_ARG;
+    if (S == 0) return MOE_OK;
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || (bias && !aligned(bias, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_route_sigmoid_grouped(logits, bias, S, E, K, n_group, n_group > 1 ? topk_group : 1,
+                                                   normalize, scale, topk_idx, topk_w,
+                                                   static_cast<cudaStream_t>(stream), current_sms()));
+}
+
 size_t moe_dispatch_layout_workspace(int S, int E, int K) {
     if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK) return 0;
     if ((int64_t)S * K >= ((int64_t)1 << 31)) return 0;

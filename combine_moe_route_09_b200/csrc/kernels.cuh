@@ -52,6 +52,10 @@ cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y
                                     void *grad_y, float *grad_w, void *grad_skip, int32_t *status,
                                     cudaStream_t st);
 
+cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                                         int topk_group, int normalize, float scale, int32_t *idx, float *w,
+                                         cudaStream_t st, int sms);
+
 cudaError_t launch_route_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w, int S,
                                   int E, int K, float *grad_logits, cudaStream_t st, int sms);
 

@@ -101,6 +101,169 @@ cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t 
     return launch_route<32>(logits, S, E, K, idx, w, st, sms);
 }
 
+// ------------------------------------------------------------------------------------------
+// Router variant: sigmoid scores, selection-only bias, group-limited top-K (the
+// DeepSeek-V3 router that "Efficient and portable mixture-of-experts
+// communication" cites; plainest reading).  exp is built from IEEE basic
+// operations -- Cody-Waite reduction with a 16-bit head of ln 2, the degree-7
+// Taylor polynomial in Horner form, two exact power-of-two factors -- and every
+// operation below is an explicit round-to-nearest intrinsic (no contraction), so
+// the selection scores are the same fp32 values the oracle computes.
+// ------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+__device__ __forceinline__ float route_exp(float x) {
+    if (x > 88.72283935546875f) return __int_as_float(0x7f800000);
+    if (x < -103.97208404541015625f) return 0.0f;
+    const float n = rintf(__fmul_rn(x, 1.44269502162933349609375f));
+    float r = __fmaf_rn(-n, 0.693145751953125f, x);
+    r = __fmaf_rn(-n, 1.428606765330187045037746429443359375e-06f, r);
+    float p = 1.9841270114e-04f;
+    p = __fmaf_rn(p, r, 1.3888889225e-03f);
+    p = __fmaf_rn(p, r, 8.3333337680e-03f);
+    p = __fmaf_rn(p, r, 4.1666667908e-02f);
+    p = __fmaf_rn(p, r, 1.6666667163e-01f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ni = (int)n;
+    const int h = ni / 2;
+    return __fmul_rn(__fmul_rn(p, pow2i(h)), pow2i(ni - h));
+}
+
+__device__ __forceinline__ float route_sigmoid(float l) {
+    return __fdiv_rn(1.0f, __fadd_rn(1.0f, route_exp(-l)));
+}
+
+template <int NPER>
+__global__ void __launch_bounds__(256)
+    route_sigmoid_grouped_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int S, int E,
+                                 int K, int n_group, int topk_group, int normalize, float scale,
+                                 int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    const int gsize = E / n_group;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
+        const float *row = logits + (size_t)t * E;
+        float sv[NPER], cv[NPER];
+        int gid[NPER];  // group of each held expert; n_group for lanes past E
+#pragma unroll
+        for (int j = 0; j < NPER; ++j) {
+            const int e = lane + 32 * j;
+            gid[j] = e < E ? e / gsize : n_group;
+            sv[j] = 0.f;
+            cv[j] = __int_as_float(0xff800000);  // -inf: not an expert
+            if (e < E) {
+                sv[j] = route_sigmoid(__ldg(row + e));
+                cv[j] = bias ? __fadd_rn(sv[j], __ldg(bias + e)) : sv[j];
+            }
+        }
+        // ---- groups: score = largest + second largest selection score ----
+        uint32_t gmask = 0xffffffffu;
+        if (n_group > 1) {
+            float my_gs = 0.f;
+            for (int g = 0; g < n_group; ++g) {
+                float a1 = __int_as_float(0xff800000), a2 = a1;
+#pragma unroll
+                for (int j = 0; j < NPER; ++j) {
+                    if (gid[j] == g) {
+                        const float v = cv[j];
+                        a2 = fmaxf(a2, fminf(a1, v));
+                        a1 = fmaxf(a1, v);
+                    }
+                }
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) {
+                    const float b1 = __shfl_xor_sync(FULL, a1, m), b2 = __shfl_xor_sync(FULL, a2, m);
+                    const float n2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+                    a1 = fmaxf(a1, b1);
+                    a2 = n2;
+                }
+                if (lane == g) my_gs = __fadd_rn(a1, a2);
+            }
+            // keep the topk_group best groups (ties: lower group)
+            bool taken = false;
+            for (int r = 0; r < topk_group; ++r) {
+                const uint32_t key = (lane < n_group && !taken) ? ordered_bits(my_gs) : 0u;
+                const uint32_t best = __reduce_max_sync(FULL, key);
+                const uint32_t win = __reduce_min_sync(FULL, (key == best && lane < n_group && !taken) ? (uint32_t)lane : 0xffffffffu);
+                if ((uint32_t)lane == win) taken = true;
+            }
+            gmask = __ballot_sync(FULL, taken);
+        }
+        // ---- top-K of the selection score over the experts of the kept groups ----
+        uint32_t key[NPER];
+#pragma unroll
+        for (int j = 0; j < NPER; ++j) {
+            key[j] = (gid[j] < n_group && ((gmask >> gid[j]) & 1u)) ? ordered_bits(cv[j]) : 0u;
+        }
+        float my_s = 0.f;
+        int my_e = 0;
+        for (int k = 0; k < K; ++k) {
+            uint32_t m = key[0];
+#pragma unroll
+            for (int j = 1; j < NPER; ++j) m = max(m, key[j]);
+            const uint32_t best = __reduce_max_sync(FULL, m);
+            uint32_t cand = 0xffffffffu;
+#pragma unroll
+            for (int j = NPER - 1; j >= 0; --j) cand = key[j] == best ? (uint32_t)(lane + 32 * j) : cand;
+            const uint32_t win = __reduce_min_sync(FULL, cand);
+            float own = 0.f;  // the winner's unbiased score, from its owner lane
+#pragma unroll
+            for (int j = 0; j < NPER; ++j) own = (uint32_t)(lane + 32 * j) == win ? sv[j] : own;
+            const float s_win = __shfl_sync(FULL, own, (int)(win & 31u));
+            if (lane == k) {
+                my_s = s_win;
+                my_e = (int)win;
+            }
+#pragma unroll
+            for (int j = 0; j < NPER; ++j) key[j] = (uint32_t)(lane + 32 * j) == win ? 0u : key[j];
+        }
+        float sum = 0.f;  // in k order, as the oracle
+        for (int k = 0; k < K; ++k) sum = __fadd_rn(sum, __shfl_sync(FULL, my_s, k));
+        if (lane < K) {
+            const float v = normalize ? __fdiv_rn(my_s, sum) : my_s;
+            topk_idx[(size_t)t * K + lane] = my_e;
+            topk_w[(size_t)t * K + lane] = __fmul_rn(v, scale);
+        }
+    }
+}
+
+template <int NPER>
+static cudaError_t launch_sg(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                             int topk_group, int normalize, float scale, int32_t *idx, float *w, cudaStream_t st,
+                             int sms) {
+    const int threads = 256;
+    int blocks = (S + 7) / 8;
+    if (blocks > sms * 8) blocks = sms * 8;
+    if (blocks < 1) blocks = 1;
+    static KernelSlots<decltype(&route_sigmoid_grouped_kernel<NPER>)> slots;
+    int n_sms = 0, per_sm = 0;
+    const cudaError_t e = slots.prepare(&route_sigmoid_grouped_kernel<NPER>, threads, 0, &n_sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(route_sigmoid_grouped_kernel<NPER>, dim3(blocks), dim3(threads), 0, st, logits, bias, S, E,
+                      K, n_group, topk_group, normalize, scale, idx, w);
+}
+
+cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                                         int topk_group, int normalize, float scale, int32_t *idx, float *w,
+                                         cudaStream_t st, int sms) {
+    const int nper = (E + 31) / 32;
+#define MOE_SG(N) return launch_sg<N>(logits, bias, S, E, K, n_group, topk_group, normalize, scale, idx, w, st, sms)
+    if (nper <= 1) MOE_SG(1);
+    if (nper <= 2) MOE_SG(2);
+    if (nper <= 4) MOE_SG(4);
+    if (nper <= 8) MOE_SG(8);
+    if (nper <= 12) MOE_SG(12);
+    if (nper <= 16) MOE_SG(16);
+    if (nper <= 24) MOE_SG(24);
+    MOE_SG(32);
+#undef MOE_SG
+}
+
 // Backward through the gating softmax: for the selected experts
 // grad_logits[t, e_k] = w_k (gw_k - sum_j w_j gw_j), 0 for the others.  One warp
 // per token: the dense row is zeroed, then lanes k < K write their entries

@@ -109,6 +109,29 @@ MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *to
                    void *stream);
 
 /*
+ * Router variant: sigmoid scores, a selection-only bias and group-limited
+ * top-K -- the router of the DeepSeek-V3 report, which "Efficient and portable
+ * mixture-of-experts communication" cites; the pages give no detail, so this
+ * is the plainest reading:
+ *   s_e = sigmoid(l_e);  c_e = s_e + bias_e (bias [E] fp32, or NULL: c = s)
+ *   n_group > 1: experts form n_group contiguous groups of E/n_group; a group's
+ *     score is its largest c plus its second largest c; the topk_group best
+ *     groups (ties: lower group) are kept, the others excluded
+ *   topk_idx: the K largest c among kept experts (descending; ties: lower id)
+ *   topk_w:  s_{e_k}, divided by sum_k s_{e_k} (k order) when normalize != 0,
+ *            then multiplied by scale
+ * All fp32; exp comes from IEEE basic operations (Cody-Waite reduction and a
+ * degree-7 polynomial, within 2 ulp of exp), so results are reproducible.
+ * Host checks: those of moe_route_topk, plus 1 <= n_group <= MOE_MAX_GROUPS,
+ * E % n_group == 0, and for n_group > 1: E/n_group >= 2,
+ * 1 <= topk_group <= n_group, topk_group * E / n_group >= K.
+ */
+#define MOE_MAX_GROUPS 32
+MOE_API int moe_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
+                                      int topk_group, int normalize, float scale, int32_t *topk_idx,
+                                      float *topk_w, void *stream);
+
+/*
  * Bytes of scratch memory moe_dispatch_layout needs for these sizes
  * (a host-side query; no device work).  Returns 0 for invalid sizes.
  */
