@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     moe_dispatch_backward,
     moe_dispatch_layout,
     moe_dispatch_layout_workspace,
+    moe_dispatch_route_weights,
     moe_route_topk,
     moe_route_sigmoid_grouped,
     moe_route_topk_backward,

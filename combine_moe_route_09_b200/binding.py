@@ -29,6 +29,7 @@ _P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 # name -> (restype, argtypes), the exact C signatures
 SIGNATURES = {
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_dispatch_route_weights": (_I, [_P, _P, _I, _I, _L, _P, _P, _P]),
     "moe_route_sigmoid_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _Z, _P, _P]),
@@ -119,6 +120,20 @@ def moe_route_topk(logits: torch.Tensor, K: int, topk_idx=None, topk_w=None, str
     _check("moe_route_topk", lib().moe_route_topk(_ptr(logits), S, E, K, _ptr(topk_idx), _ptr(topk_w),
                                                    _stream(stream, logits.device)))
     return topk_idx, topk_w
+
+
+def moe_dispatch_route_weights(topk_w: torch.Tensor, row_src: torch.Tensor, out=None, status=None, stream=None):
+    """Routing weights in dispatched order: out[r] = topk_w.flat[row_src[r]], 0 where row_src < 0."""
+    _dev(topk_w, "topk_w", (torch.float32,))
+    _dev(row_src, "row_src", (torch.int32,))
+    S, K = topk_w.shape
+    cap = row_src.shape[0]
+    if out is None:
+        out = torch.empty(cap, dtype=torch.float32, device=row_src.device)
+    _dev(out, "route_weights", (torch.float32,), (cap,))
+    _check("moe_dispatch_route_weights", lib().moe_dispatch_route_weights(
+        _ptr(topk_w), _ptr(row_src), S, K, cap, _ptr(out), _ptr(status), _stream(stream, row_src.device)))
+    return out
 
 
 def moe_route_sigmoid_grouped(logits: torch.Tensor, K: int, bias=None, n_group: int = 1,

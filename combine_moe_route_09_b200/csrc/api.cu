@@ -57,6 +57,18 @@ int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, 
                                         static_cast<cudaStream_t>(stream), current_sms()));
 }
 
+int moe_dispatch_route_weights(const float *topk_w, const int32_t *row_src, int S, int K, int64_t cap,
+                               float *route_weights, int32_t *status, void *stream) {
+    if (S < 0 || K < 1 || K > MOE_MAX_TOPK || cap < 0 || cap >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+    if (cap == 0) return MOE_OK;
+    if (!row_src || !route_weights || (S > 0 && !topk_w)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(row_src, 4) || !aligned(route_weights, 4) || (topk_w && !aligned(topk_w, 4)) ||
+        (status && !aligned(status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_route_weights(topk_w, row_src, (int64_t)S * K, cap, route_weights, status,
+                                           static_cast<cudaStream_t>(stream), current_sms()));
+}
+
 int moe_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
                               int topk_group, int normalize, float scale, int32_t *topk_idx, float *topk_w,
                               void *stream) {

@@ -56,6 +56,9 @@ cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias,
                                          int topk_group, int normalize, float scale, int32_t *idx, float *w,
                                          cudaStream_t st, int sms);
 
+cudaError_t launch_route_weights(const float *topk_w, const int32_t *row_src, int64_t pairs, int64_t cap,
+                                 float *out, int32_t *status, cudaStream_t st, int sms);
+
 cudaError_t launch_route_backward(const int32_t *topk_idx, const float *topk_w, const float *grad_w, int S,
                                   int E, int K, float *grad_logits, cudaStream_t st, int sms);
 

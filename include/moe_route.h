@@ -109,6 +109,21 @@ MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *to
                    void *stream);
 
 /*
+ * Routing weights in dispatched order (MoonEP developer guide, core API
+ * example: the dispatch returns each expert's rows together with their routing
+ * weights, which the combine consumes).
+ *   topk_w         [S, K] fp32, from moe_route_topk / moe_route_sigmoid_grouped
+ *   row_src        [cap] int32, from moe_dispatch_layout (pair t*K + k, or -1)
+ *   route_weights  [cap] fp32 out: topk_w[row_src[r]] where row_src[r] >= 0,
+ *                  else 0 (padding rows and unused capacity)
+ * A row_src entry >= S*K is skipped (written 0) and sets MOE_STATUS_BAD_SLOT.
+ * Host checks: S >= 0, 1 <= K <= MOE_MAX_TOPK, 0 <= cap < 2^31, 4-byte aligned
+ * pointers.  One kernel; no synchronisation; status may be NULL.
+ */
+MOE_API int moe_dispatch_route_weights(const float *topk_w, const int32_t *row_src, int S, int K, int64_t cap,
+                                       float *route_weights, int32_t *status, void *stream);
+
+/*
  * Router variant: sigmoid scores, a selection-only bias and group-limited
  * top-K -- the router of the DeepSeek-V3 report, which "Efficient and portable
  * mixture-of-experts communication" cites; the pages give no detail, so this

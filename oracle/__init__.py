@@ -60,6 +60,7 @@ def _load():
         lib.oracle_combine_backward.argtypes = [P, P, P, I, I, I, I, L, P, P, P, P, P]
         lib.oracle_dispatch_backward.argtypes = [P, I, I, I, I, L, P, P]
         lib.oracle_route_backward.argtypes = [P, P, P, I, I, I, P]
+        lib.oracle_route_weights_dispatched.argtypes = [P, P, I, I, L, P]
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -278,6 +279,18 @@ def route_backward(topk_idx, topk_w, grad_w, E: int):
     rc = _load().oracle_route_backward(_ptr(topk_idx), _ptr(topk_w), _ptr(grad_w), S, E, K, _ptr(out))
     if rc:
         raise OracleError("oracle_route_backward", rc)
+    return out
+
+
+def route_weights_dispatched(topk_w, slot_of, cap: int):
+    """Routing weights in dispatched order: float32 [cap], 0 on rows no pair fills."""
+    topk_w = _c(topk_w, np.float32)
+    slot_of = _c(slot_of, np.int32)
+    S, K = slot_of.shape
+    out = np.empty(cap, np.float32)
+    rc = _load().oracle_route_weights_dispatched(_ptr(topk_w), _ptr(slot_of), S, K, cap, _ptr(out))
+    if rc:
+        raise OracleError("oracle_route_weights_dispatched", rc)
     return out
 
 

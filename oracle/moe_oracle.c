@@ -470,6 +470,26 @@ int oracle_dispatch_backward(const void *grad_xd, int dtype, int S, int H, int K
 }
 
 /*
+ * Route weights in dispatched order (MoonEP developer guide, core API example:
+ * the dispatch also returns the routing weights of the rows it sends, which the
+ * combine consumes).  Row slot_of[t,k] of the dispatched buffer carries
+ * topk_w[t,k]; every other row of [0, cap) -- padding, unused capacity, pairs
+ * dropped for a bad slot -- carries 0.
+ */
+int oracle_route_weights_dispatched(const float *topk_w, const int32_t *slot_of, int S, int K, int64_t cap,
+                                    float *route_weights)
+{
+    if (S < 0 || K < 1 || cap < 0) return ORACLE_EINVAL;
+    for (int64_t r = 0; r < cap; ++r) route_weights[r] = 0.0f;
+    for (int t = 0; t < S; ++t)
+        for (int k = 0; k < K; ++k) {
+            int32_t s = slot_of[(size_t)t * K + k];
+            if (s >= 0 && (int64_t)s < cap) route_weights[s] = topk_w[(size_t)t * K + k];
+        }
+    return ORACLE_OK;
+}
+
+/*
  * Backward of oracle_route_topk through the gating softmax.  The weights are
  * the softmax of the K selected logits, so for the selected experts
  *     grad_logits[t, e_k] = w_k * (gw_k - sum_j w_j gw_j)

@@ -129,3 +129,30 @@ def test_layout_errors(oracle_lib):
     with pytest.raises(oracle_lib.OracleError) as e:
         oracle_lib.layout(idx, 4, 3, 0)  # E % R != 0
     assert e.value.rc == oracle_lib.EINVAL
+
+
+@pytest.mark.parametrize("name,S", [("1", 128), ("2", 512), ("5", 700)])
+def test_route_weights_dispatched(oracle_lib, name, S):
+    """Row r of the dispatched order carries the weight of the pair row_src[r] names (read
+    through row_src, the other direction of the layout); rows no pair fills carry 0; per
+    expert, the rows' weights add up to the weights of the tokens routed there (bincount)."""
+    w = synth.WORKLOADS[name].replace(S=S)
+    idx, wt = oracle_lib.route_topk(synth.logits(w), w.K)
+    lay = oracle_lib.layout(idx, w.E, w.R, w.P)
+    rw = oracle_lib.route_weights_dispatched(wt, lay["slot_of"], lay["cap"])
+    src = lay["row_src"]
+    valid = src >= 0
+    np.testing.assert_array_equal(rw[valid], wt.reshape(-1)[src[valid]])
+    assert np.all(rw[~valid] == 0)
+    seg = np.repeat(np.arange(w.E), np.diff(lay["offsets"]))
+    per_expert = np.bincount(seg, weights=rw[:lay["offsets"][-1]].astype(np.float64), minlength=w.E)
+    ref = np.bincount(idx.reshape(-1), weights=wt.reshape(-1).astype(np.float64), minlength=w.E)
+    np.testing.assert_allclose(per_expert, ref, rtol=1e-12, atol=0)
+
+
+def test_route_weights_dispatched_worked_example(oracle_lib):
+    # 3 tokens, K = 2, hand-placed slots in a capacity of 8 (slot -1: pair dropped)
+    slot_of = np.array([[4, 0], [1, -1], [7, 2]], np.int32)
+    wt = np.array([[0.6, 0.4], [0.9, 0.1], [0.5, 0.5]], np.float32)
+    rw = oracle_lib.route_weights_dispatched(wt, slot_of, 8)
+    assert rw.tolist() == [np.float32(0.4), np.float32(0.9), 0.5, 0.0, np.float32(0.6), 0.0, 0.0, 0.5]
