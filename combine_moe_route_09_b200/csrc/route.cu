@@ -136,71 +136,89 @@ __device__ __forceinline__ float route_sigmoid(float l) {
     return __fdiv_rn(1.0f, __fadd_rn(1.0f, route_exp(-l)));
 }
 
+// One warp per token; lane holds experts e = lane + 32 j (j < NPER).  The
+// warp also keeps the row's scores in its own shared-memory slice, [E]
+// selection scores then [E] sigmoid scores, so that (1) the group scores are
+// scanned by LPG lanes per group (LPG = 32 / n_group rounded down to a power
+// of two) followed by an xor merge of (largest, second largest), and (2) the
+// winner's sigmoid score is one broadcast shared load.
+constexpr int SG_WARPS = 8;
+
 template <int NPER>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(SG_WARPS * 32)
     route_sigmoid_grouped_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int S, int E,
                                  int K, int n_group, int topk_group, int normalize, float scale,
                                  int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+    extern __shared__ float sg_smem[];
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
+    float *const cs = sg_smem + (size_t)wib * 2 * E;  // selection scores of the warp's row
+    float *const ss = cs + E;                         // sigmoid scores
     const int warps = (gridDim.x * blockDim.x) >> 5;
     const int gsize = E / n_group;
+    int lpg = 1;  // lanes per group
+    while (lpg * 2 * n_group <= 32) lpg *= 2;
+    const int my_g = lane / lpg, my_sub = lane - my_g * lpg;
+    const float NEG_INF = __int_as_float(0xff800000);
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
         const float *row = logits + (size_t)t * E;
-        float sv[NPER], cv[NPER];
-        int gid[NPER];  // group of each held expert; n_group for lanes past E
+        float cv[NPER];
 #pragma unroll
         for (int j = 0; j < NPER; ++j) {
             const int e = lane + 32 * j;
-            gid[j] = e < E ? e / gsize : n_group;
-            sv[j] = 0.f;
-            cv[j] = __int_as_float(0xff800000);  // -inf: not an expert
+            cv[j] = NEG_INF;  // not an expert
             if (e < E) {
-                sv[j] = route_sigmoid(__ldg(row + e));
-                cv[j] = bias ? __fadd_rn(sv[j], __ldg(bias + e)) : sv[j];
+                // sigmoid = 1 / (1 + exp(-l)): the correctly rounded reciprocal is the
+                // correctly rounded quotient 1 / d
+                const float sg = __frcp_rn(__fadd_rn(1.0f, route_exp(-__ldg(row + e))));
+                cv[j] = bias ? __fadd_rn(sg, __ldg(bias + e)) : sg;
+                cs[e] = cv[j];
+                ss[e] = sg;
             }
         }
+        __syncwarp();
         // ---- groups: score = largest + second largest selection score ----
-        uint32_t gmask = 0xffffffffu;
+        uint32_t keep = 0xffffffffu;  // bit (g * lpg) set: group g kept
         if (n_group > 1) {
-            float my_gs = 0.f;
-            for (int g = 0; g < n_group; ++g) {
-                float a1 = __int_as_float(0xff800000), a2 = a1;
-#pragma unroll
-                for (int j = 0; j < NPER; ++j) {
-                    if (gid[j] == g) {
-                        const float v = cv[j];
-                        a2 = fmaxf(a2, fminf(a1, v));
-                        a1 = fmaxf(a1, v);
-                    }
+            float a1 = NEG_INF, a2 = NEG_INF;
+            if (my_g < n_group) {
+                const float *grp = cs + my_g * gsize;
+                for (int i = my_sub; i < gsize; i += lpg) {
+                    const float v = grp[i];
+                    a2 = fmaxf(a2, fminf(a1, v));
+                    a1 = fmaxf(a1, v);
                 }
-#pragma unroll
-                for (int m = 16; m > 0; m >>= 1) {
-                    const float b1 = __shfl_xor_sync(FULL, a1, m), b2 = __shfl_xor_sync(FULL, a2, m);
-                    const float n2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
-                    a1 = fmaxf(a1, b1);
-                    a2 = n2;
-                }
-                if (lane == g) my_gs = __fadd_rn(a1, a2);
             }
-            // keep the topk_group best groups (ties: lower group)
+            for (int m = 1; m < lpg; m <<= 1) {
+                const float b1 = __shfl_xor_sync(FULL, a1, m), b2 = __shfl_xor_sync(FULL, a2, m);
+                const float n2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+                a1 = fmaxf(a1, b1);
+                a2 = n2;
+            }
+            const bool leader = my_g < n_group && my_sub == 0;
+            const uint32_t gkey = leader ? ordered_bits(__fadd_rn(a1, a2)) : 0u;
             bool taken = false;
+            // keep the topk_group best groups (ties: lower group = lower lane)
             for (int r = 0; r < topk_group; ++r) {
-                const uint32_t key = (lane < n_group && !taken) ? ordered_bits(my_gs) : 0u;
+                const uint32_t key = (leader && !taken) ? gkey : 0u;
                 const uint32_t best = __reduce_max_sync(FULL, key);
-                const uint32_t win = __reduce_min_sync(FULL, (key == best && lane < n_group && !taken) ? (uint32_t)lane : 0xffffffffu);
+                const uint32_t win =
+                    __reduce_min_sync(FULL, (leader && !taken && gkey == best) ? (uint32_t)lane : 0xffffffffu);
                 if ((uint32_t)lane == win) taken = true;
             }
-            gmask = __ballot_sync(FULL, taken);
+            keep = __ballot_sync(FULL, taken);
         }
         // ---- top-K of the selection score over the experts of the kept groups ----
         uint32_t key[NPER];
 #pragma unroll
         for (int j = 0; j < NPER; ++j) {
-            key[j] = (gid[j] < n_group && ((gmask >> gid[j]) & 1u)) ? ordered_bits(cv[j]) : 0u;
+            const int e = lane + 32 * j;
+            bool ok = e < E;
+            if (n_group > 1 && ok) ok = (keep >> ((e / gsize) * lpg)) & 1u;
+            key[j] = ok ? ordered_bits(cv[j]) : 0u;
         }
-        float my_s = 0.f;
         int my_e = 0;
         for (int k = 0; k < K; ++k) {
             uint32_t m = key[0];
@@ -211,17 +229,12 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int j = NPER - 1; j >= 0; --j) cand = key[j] == best ? (uint32_t)(lane + 32 * j) : cand;
             const uint32_t win = __reduce_min_sync(FULL, cand);
-            float own = 0.f;  // the winner's unbiased score, from its owner lane
-#pragma unroll
-            for (int j = 0; j < NPER; ++j) own = (uint32_t)(lane + 32 * j) == win ? sv[j] : own;
-            const float s_win = __shfl_sync(FULL, own, (int)(win & 31u));
-            if (lane == k) {
-                my_s = s_win;
-                my_e = (int)win;
-            }
+            if (lane == k) my_e = (int)win;
 #pragma unroll
             for (int j = 0; j < NPER; ++j) key[j] = (uint32_t)(lane + 32 * j) == win ? 0u : key[j];
         }
+        // the winners' unbiased scores (an id past E only from NaN logits: read as 0)
+        const float my_s = (lane < K && (unsigned)my_e < (unsigned)E) ? ss[my_e] : 0.f;
         float sum = 0.f;  // in k order, as the oracle
         for (int k = 0; k < K; ++k) sum = __fadd_rn(sum, __shfl_sync(FULL, my_s, k));
         if (lane < K) {
@@ -229,6 +242,7 @@ __global__ void __launch_bounds__(256)
             topk_idx[(size_t)t * K + lane] = my_e;
             topk_w[(size_t)t * K + lane] = __fmul_rn(v, scale);
         }
+        __syncwarp();  // the slice is rewritten by the warp's next token
     }
 }
 
@@ -236,16 +250,18 @@ template <int NPER>
 static cudaError_t launch_sg(const float *logits, const float *bias, int S, int E, int K, int n_group,
                              int topk_group, int normalize, float scale, int32_t *idx, float *w, cudaStream_t st,
                              int sms) {
-    const int threads = 256;
-    int blocks = (S + 7) / 8;
-    if (blocks > sms * 8) blocks = sms * 8;
-    if (blocks < 1) blocks = 1;
+    const int threads = SG_WARPS * 32;
+    const size_t smem = (size_t)SG_WARPS * 2 * E * sizeof(float);
     static KernelSlots<decltype(&route_sigmoid_grouped_kernel<NPER>)> slots;
     int n_sms = 0, per_sm = 0;
-    const cudaError_t e = slots.prepare(&route_sigmoid_grouped_kernel<NPER>, threads, 0, &n_sms, &per_sm);
+    const cudaError_t e = slots.prepare(&route_sigmoid_grouped_kernel<NPER>, threads, smem, &n_sms, &per_sm);
     if (e != cudaSuccess) return e;
-    return launch_pdl(route_sigmoid_grouped_kernel<NPER>, dim3(blocks), dim3(threads), 0, st, logits, bias, S, E,
-                      K, n_group, topk_group, normalize, scale, idx, w);
+    long long blocks = ((long long)S + SG_WARPS - 1) / SG_WARPS;
+    const long long resident = (long long)n_sms * (per_sm > 0 ? per_sm : 1);
+    if (blocks > resident) blocks = resident;
+    if (blocks < 1) blocks = 1;
+    return launch_pdl(route_sigmoid_grouped_kernel<NPER>, dim3((unsigned)blocks), dim3(threads), smem, st, logits,
+                      bias, S, E, K, n_group, topk_group, normalize, scale, idx, w);
 }
 
 cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias, int S, int E, int K, int n_group,
