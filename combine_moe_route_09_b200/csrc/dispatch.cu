@@ -141,8 +141,14 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
 // FP8 e4m3, 128-channel blocks
 // ------------------------------------------------------------------------------------------
 
+#ifndef MOE_DQ_STAGE_BUDGET
+#define MOE_DQ_STAGE_BUDGET (48 * 1024)
+#endif
+#ifndef MOE_DQ_MIN_CTAS
+#define MOE_DQ_MIN_CTAS 1
+#endif
 constexpr int DQ_MAX_STAGES = 8;
-constexpr int DQ_STAGE_BUDGET = 48 * 1024;                   // bytes of input ring per CTA
+constexpr int DQ_STAGE_BUDGET = MOE_DQ_STAGE_BUDGET;         // bytes of input ring per CTA
 constexpr int DQ_CONSUMER_WARPS = 4;
 constexpr int DQ_CONSUMERS = DQ_CONSUMER_WARPS * 32;
 constexpr int DQ_THREADS = DQ_CONSUMERS + 32;
@@ -184,13 +190,15 @@ __device__ __forceinline__ float scale_of(float amax) {
 // of x * r with r = 1/s correctly rounded (P. Markstein, "Computation of
 // elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
 // Dev. 34(1), 1990): with r = RN(1/s), q0 = RN(x r) and the remainder
-// e = x - q0 s exact (one fma), RN(q0 + e r) = RN(x / s).  The theorem is
-// about non-zero quotients; for x = -0 the correction yields +0, so the sign
-// of x (the sign of x / s, as s > 0) is copied onto the result.
+// e = x - q0 s exact (one fma), RN(q0 + e r) = RN(x / s).  The remainder is
+// formed negated, n = q0 s - x, and the quotient as RN(q0 + (-n) r): the same
+// values for x != 0, and for x = -0 the sums (-0) + (+0) -> +0 and
+// (-0) + (-0) -> -0 keep the sign of the zero quotient (three operations, the
+// negations being free operand modifiers).
 __device__ __forceinline__ float div_markstein(float x, float s, float r) {
     const float q0 = __fmul_rn(x, r);
-    const float e = __fmaf_rn(-q0, s, x);
-    return copysignf(__fmaf_rn(e, r, q0), x);
+    const float n = __fmaf_rn(q0, s, -x);
+    return __fmaf_rn(-n, r, q0);
 }
 
 // 16 values -> 16 e4m3 codes (value i in byte i), given the block scale s.
@@ -229,7 +237,7 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
 
 // KT: K known at compile time (0 = runtime K).
 template <bool IN_F32, int KT>
-__global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args a) {
+__global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kernel(const Fp8Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     // layout: [stages][header (K slots) | bpc*128*esz input bytes] | barriers
     const int NS = a.stages;

@@ -503,6 +503,217 @@ __global__ void __launch_bounds__(LT_THREADS)
         row_src[r] = -1;
 }
 
+// ------------------------------------------------------------------------------------------
+// Cluster layout: up to LC_MAX_CTAS tiles of LC_TILE pairs, one CTA each, all
+// in one thread-block cluster.  Each CTA ranks its tile (as above, with 32
+// warps), keeps the tile histogram in its own shared memory, and after one
+// hardware cluster barrier reads the other CTAs' histograms through
+// distributed shared memory: the per-expert totals and the counts of the tiles
+// below it.  No global scratch, no atomics, no spin-wait.  A second cluster
+// barrier (arrive after the remote reads, wait before exit) keeps every CTA's
+// shared memory alive until the others have read it.
+// ------------------------------------------------------------------------------------------
+
+constexpr int LC_WARPS = 32;
+constexpr int LC_THREADS = LC_WARPS * 32;
+constexpr int LC_ITEMS = 4;
+constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // 4096 pairs
+constexpr int LC_MAX_CTAS = 8;                 // portable cluster size
+
+__global__ void __launch_bounds__(LC_THREADS)
+    layout_cluster_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P, int64_t cap,
+                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                          int32_t *__restrict__ rank_offsets, int32_t *__restrict__ slot_of,
+                          int32_t *__restrict__ row_src, int32_t *status) {
+    extern __shared__ __align__(16) uint8_t lc_smem[];
+    int *thist = reinterpret_cast<int *>(lc_smem);             // [E] this tile's counts (read cluster-wide)
+    int *s_tot = thist + E;                                     // [E] totals
+    int *s_base = s_tot + E;                                    // [E] first row of this tile's pairs, per expert
+    int *s_off = s_base + E;                                    // [E + 1] padded offsets
+    uint16_t *whist = reinterpret_cast<uint16_t *>(s_off + E + 1 + 3);  // [LC_WARPS][E]
+    __shared__ int s_wsum[LC_WARPS];
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int C = gridDim.x;
+    const uint32_t me = cluster_ctarank();
+    const int tile = blockIdx.x;
+    for (int i = tid; i < LC_WARPS * E; i += LC_THREADS) whist[i] = 0;
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    // ---- rank this CTA's pairs: warp w takes LC_ITEMS consecutive chunks of 32 ----
+    const unsigned lt = lanemask_lt();
+    int my_e[LC_ITEMS], my_r[LC_ITEMS];
+    int ev[LC_ITEMS];
+#pragma unroll
+    for (int it = 0; it < LC_ITEMS; ++it) {
+        const int p = tile * LC_TILE + (w * LC_ITEMS + it) * 32 + lane;
+        ev[it] = p < npairs ? __ldcg(topk_idx + p) : -1;  // through L2: written by the previous kernel
+    }
+    bool bad = false;
+#pragma unroll
+    for (int it = 0; it < LC_ITEMS; ++it) {
+        const int p = tile * LC_TILE + (w * LC_ITEMS + it) * 32 + lane;
+        int e = ev[it];
+        if (p < npairs && (e < 0 || e >= E)) {
+            bad = true;
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(FULL, e);
+        const int before = e >= 0 ? (int)whist[w * E + e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
+        __syncwarp();
+        my_e[it] = e;
+        my_r[it] = before + __popc(peers & lt);
+    }
+    if (bad) set_status(status, MOE_STATUS_BAD_INDEX);
+    __syncthreads();
+    // per-warp counts -> exclusive prefix over warps; the tile's total per expert
+    for (int e = tid; e < E; e += LC_THREADS) {
+        int run = 0;
+#pragma unroll 8
+        for (int ww = 0; ww < LC_WARPS; ++ww) {
+            const int c = whist[ww * E + e];
+            whist[ww * E + e] = (uint16_t)run;
+            run += c;
+        }
+        thist[e] = run;
+    }
+    cluster_arrive();
+    cluster_wait();  // every tile histogram of the cluster is complete and visible
+
+    // ---- totals and the count of the tiles below this one, from all CTAs' thist ----
+    const uint32_t th = smem_addr(thist);
+    for (int e = tid; e < E; e += LC_THREADS) {
+        int all = 0, below = 0;
+        for (int c = 0; c < C; ++c) {
+            const int v = ld_cluster_s32(cluster_map(th + 4u * e, (uint32_t)c));
+            all += v;
+            below += (uint32_t)c < me ? v : 0;
+        }
+        s_tot[e] = all;
+        s_base[e] = below;
+    }
+    cluster_arrive();  // done reading the others' shared memory (waited for before exit)
+    __syncthreads();
+
+    // ---- exclusive scan of the padded counts over experts (one expert per thread) ----
+    const int pc = tid < E ? pad_count(s_tot[tid], P) : 0;
+    int incl = pc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = s_wsum[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(FULL, v, off);
+            if (lane >= off) v += o;
+        }
+        s_wsum[lane] = v;  // inclusive over warps
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int off = incl - pc + (w > 0 ? s_wsum[w - 1] : 0);
+        s_off[tid] = off;
+        s_base[tid] += off;
+    }
+    if (tid == 0) s_off[E] = s_wsum[LC_WARPS - 1];
+    __syncthreads();
+    if (me == 0) {
+        for (int e = tid; e <= E; e += LC_THREADS) offsets[e] = s_off[e];
+        for (int e = tid; e < E; e += LC_THREADS) counts[e] = s_tot[e];
+        const int Eloc = E / R;
+        for (int r = tid; r <= R; r += LC_THREADS) rank_offsets[r] = s_off[r * Eloc];
+        if (tid == 0 && (int64_t)s_off[E] > cap) set_status(status, MOE_STATUS_OVERFLOW);
+    }
+
+    // ---- slots ----
+    bool over = false;
+#pragma unroll
+    for (int it = 0; it < LC_ITEMS; ++it) {
+        const int p = tile * LC_TILE + (w * LC_ITEMS + it) * 32 + lane;
+        if (p >= npairs) continue;
+        const int e = my_e[it];
+        int sl = -1;
+        if (e >= 0) {
+            sl = s_base[e] + whist[w * E + e] + my_r[it];
+            if ((int64_t)sl >= cap) {
+                sl = -1;
+                over = true;
+            }
+        }
+        slot_of[p] = sl;
+        if (sl >= 0) row_src[sl] = p;
+    }
+    if (over) set_status(status, MOE_STATUS_OVERFLOW);
+
+    // ---- padding rows (one warp per expert) and rows past the layout ----
+    const int gw = tile * LC_WARPS + w, nw = C * LC_WARPS;
+    for (int e = gw; e < E; e += nw) {
+        const int64_t lo = (int64_t)s_off[e] + s_tot[e];
+        int64_t hi = s_off[e + 1];
+        if (hi > cap) hi = cap;
+        for (int64_t r = lo + lane; r < hi; r += 32) row_src[r] = -1;
+    }
+    for (int64_t r = (int64_t)s_off[E] + (int64_t)tile * LC_THREADS + tid; r < cap; r += (int64_t)C * LC_THREADS)
+        row_src[r] = -1;
+    cluster_wait();  // the other CTAs have finished reading this CTA's thist
+}
+
+static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap,
+                                         int32_t *counts, int32_t *offsets, int32_t *rank_offsets,
+                                         int32_t *slot_of, int32_t *row_src, int32_t *status, cudaStream_t st,
+                                         bool *launched) {
+    *launched = false;
+    const int C = (npairs + LC_TILE - 1) / LC_TILE;
+    if (C < 1 || C > LC_MAX_CTAS) return cudaSuccess;  // not launched
+    const size_t smem = (size_t)(4 * E + 4) * sizeof(int) + (size_t)LC_WARPS * E * sizeof(uint16_t);
+    static KernelSlots<decltype(&layout_cluster_kernel)> slots;
+    int sms = 0, per_sm = 0;
+    cudaError_t e = slots.prepare(&layout_cluster_kernel, LC_THREADS, smem, &sms, &per_sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaSuccess;
+    static int pdl_ok = 1, cluster_ok = 1;
+    if (!cluster_ok) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C);
+    cfg.blockDim = dim3(LC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_ok ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, topk_idx, npairs, E, R, P, cap, counts, offsets,
+                           rank_offsets, slot_of, row_src, status);
+    if (e != cudaSuccess && pdl_ok) {
+        (void)cudaGetLastError();  // the pair was refused: launch without PDL from now on
+        pdl_ok = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, topk_idx, npairs, E, R, P, cap, counts, offsets,
+                               rank_offsets, slot_of, row_src, status);
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // no cluster launch here: the other paths from now on
+        cluster_ok = 0;
+        return cudaSuccess;
+    }
+    *launched = true;
+    return cudaSuccess;
+}
+
 static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap, int T,
                                        int32_t *hist, LayoutHeader *hdr, int32_t *counts, int32_t *offsets,
                                        int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src, int32_t *status,
@@ -553,6 +764,10 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
     bool launched = false;
+    cudaError_t ce = launch_layout_cluster(topk_idx, npairs, E, R, P, cap, counts, offsets, rank_offsets, slot_of,
+                                           row_src, status, st, &launched);
+    if (ce != cudaSuccess) return ce;
+    if (launched) return cudaSuccess;
     cudaError_t fe = launch_layout_fused(topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts, offsets,
                                          rank_offsets, slot_of, row_src, status, st, &launched);
     if (fe != cudaSuccess) return fe;

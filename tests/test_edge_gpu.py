@@ -285,6 +285,10 @@ def test_fp8_quotients_near_rounding_midpoints(in_bf16):
     (8192, 1024, 32, 8, 16),   # T*E above the fused layout's scan bound: the two-kernel layout
     (150000, 64, 8, 8, 128),   # more tiles than co-resident CTAs: several tiles per CTA (fused)
     (20000, 512, 8, 4, 0),     # mid-size fused
+    (1024, 1024, 32, 8, 16),   # cluster layout: 8 CTAs of 4096 pairs, the largest E
+    (4095, 256, 8, 8, 0),      # cluster layout, ragged last tile
+    (4097, 256, 8, 8, 128),    # one tile past the cluster layout's bound: fused
+    (3, 7, 2, 1, 5),           # cluster of one CTA, E not a multiple of 32
 ])
 def test_layout_paths_large(S, E, K, R, P):
     rng = np.random.default_rng(S + E)
