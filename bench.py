@@ -524,7 +524,8 @@ def run_backward(args, w, rank, world, local_rank):
         "config": workload_config(w, world), "phases": phases,
         "roofline": {"kernel": "combine_bwd_kernel", "bound": "hbm", "achieved": cb["gb_s"], "peak": peak,
                      "unit": "GB/s", "frac": cb["gb_s"] / peak, "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": ab["combine_backward"], "traffic": None},
+                     "algorithmic_bytes_per_launch": ab["combine_backward"],
+                     "traffic": recorded_traffic("combine_bwd.cu", w.name)},
         "gpu_launches": K * 3, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -583,7 +584,8 @@ def run_fp8_combine(args, w, rank, world, local_rank):
     print(json.dumps({"mode": "fp8_combine", "metric": "combine over FP8 expert outputs, tokens/s, 1 GPU",
                       "value": S / (ms * 1e-3), "unit": "tokens/s", "us_per_call": ms * 1e3,
                       "algorithmic_bytes": nbytes, "gb_s": gbs, "frac_of_peak": gbs / peak,
-                      "peak_source": peak_kind, "config": workload_config(w, world), "clocks": clocks,
+                      "peak_source": peak_kind, "traffic": recorded_traffic("combine_fp8.cu", w.name),
+                      "config": workload_config(w, world), "clocks": clocks,
                       "steps": K, "warmup": args.warmup}), flush=True)
 
 
@@ -604,13 +606,22 @@ def run_router(args, w, rank, world, local_rank):
     idx = torch.empty((w.S, w.K), dtype=torch.int32, device=device)
     wt = torch.empty((w.S, w.K), dtype=torch.float32, device=device)
     n_group = 8 if w.E % 8 == 0 and w.E // 8 >= 2 and 4 * (w.E // 8) >= w.K else 1
+    # the layout of the softmax router's choice, for the routing weights in dispatched order
+    from combine_moe_route_09_b200.buffer import MoeBuffer
+
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, device=device)
+    buf.route(logits)
+    lay = buf.plan()
+    rw = torch.empty(buf.cap, dtype=torch.float32, device=device)
     calls = {
         "route_topk_softmax": lambda: B.moe_route_topk(logits, w.K, topk_idx=idx, topk_w=wt),
+        "route_weights_dispatched": lambda: B.moe_dispatch_route_weights(buf.topk_w, lay.row_src, out=rw),
         "route_sigmoid_grouped": lambda: B.moe_route_sigmoid_grouped(
             logits, w.K, bias=bias, n_group=n_group, topk_group=4 if n_group > 1 else 1, normalize=True,
             scale=2.5, topk_idx=idx, topk_w=wt),
     }
     nbytes = w.S * w.E * 4 + w.S * w.K * 8 + (w.E * 4)
+    rw_bytes = buf.cap * 8 + w.S * w.K * 4  # row_src read, weights written, topk_w gathered
     peak, peak_kind = read_peak_hbm()
     res = {}
     sampler = ClockSampler(local_rank)
@@ -626,7 +637,7 @@ def run_router(args, w, rank, world, local_rank):
         ev1.record()
         torch.cuda.synchronize()
         us = ev0.elapsed_time(ev1) * 1e3 / args.steps
-        gbs = nbytes / (us * 1e-6) / 1e9
+        gbs = (rw_bytes if name == "route_weights_dispatched" else nbytes) / (us * 1e-6) / 1e9
         res[name] = {"us_per_call": us, "tokens_per_s": w.S / (us * 1e-6), "gb_s": gbs, "frac_of_peak": gbs / peak}
     clocks = sampler.stop()
     if rank != 0:

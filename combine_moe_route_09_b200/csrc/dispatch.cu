@@ -340,9 +340,15 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
                         f[u][4 * l + 3] = __uint_as_float(v.w);
                     }
                 } else {
+                    // Lanes sit 32 bytes apart, so a quarter-warp's first halves would
+                    // share 16 banks; lanes 4-7 (mod 8) read their upper half first,
+                    // which puts the eight 16-byte reads of each phase on distinct banks.
+                    const uint32_t sw = (uint32_t)(lane >> 2) & 1u;
+                    const U4 a0 = lds128(src + 16u * sw), a1 = lds128(src + 16u * (sw ^ 1u));
+                    const U4 v2[2] = {sw ? a1 : a0, sw ? a0 : a1};
 #pragma unroll
                     for (int l = 0; l < 2; ++l) {
-                        const U4 v = lds128(src + 16u * l);
+                        const U4 &v = v2[l];
                         f[u][8 * l + 0] = bf16lo(v.x); f[u][8 * l + 1] = bf16hi(v.x);
                         f[u][8 * l + 2] = bf16lo(v.y); f[u][8 * l + 3] = bf16hi(v.y);
                         f[u][8 * l + 4] = bf16lo(v.z); f[u][8 * l + 5] = bf16hi(v.z);

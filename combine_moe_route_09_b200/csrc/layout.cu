@@ -570,16 +570,35 @@ __global__ void __launch_bounds__(LC_THREADS)
     }
     if (bad) set_status(status, MOE_STATUS_BAD_INDEX);
     __syncthreads();
-    // per-warp counts -> exclusive prefix over warps; the tile's total per expert
-    for (int e = tid; e < E; e += LC_THREADS) {
-        int run = 0;
-#pragma unroll 8
-        for (int ww = 0; ww < LC_WARPS; ++ww) {
-            const int c = whist[ww * E + e];
-            whist[ww * E + e] = (uint16_t)run;
-            run += c;
+    // per-warp counts -> exclusive prefix over warps, and the tile's total per
+    // expert: tpe consecutive lanes share an expert, each summing LC_WARPS / tpe
+    // warps, then an exclusive scan across those lanes (shuffles)
+    int tpe = 1;
+    while (tpe < 32 && tpe * 2 * E <= LC_THREADS) tpe *= 2;
+    {
+        const int wpt = LC_WARPS / tpe, sub = lane & (tpe - 1), epw = 32 / tpe;
+        const int w0 = sub * wpt;
+        for (int e0 = w * epw; e0 < E; e0 += LC_WARPS * epw) {  // warp-uniform trip count
+            const int e = e0 + lane / tpe;
+            const bool ok = e < E;
+            int part = 0;
+            if (ok)
+                for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * E + e];
+            int incl = part;  // inclusive scan over the tpe lanes of this expert
+            for (int off = 1; off < tpe; off <<= 1) {
+                const int o = __shfl_up_sync(FULL, incl, off, tpe);
+                if (sub >= off) incl += o;
+            }
+            if (ok) {
+                int run = incl - part;
+                for (int ww = w0; ww < w0 + wpt; ++ww) {
+                    const int c = whist[ww * E + e];
+                    whist[ww * E + e] = (uint16_t)run;
+                    run += c;
+                }
+                if (sub == tpe - 1) thist[e] = incl;
+            }
         }
-        thist[e] = run;
     }
     cluster_arrive();
     cluster_wait();  // every tile histogram of the cluster is complete and visible
@@ -587,16 +606,20 @@ __global__ void __launch_bounds__(LC_THREADS)
     // ---- totals and the count of the tiles below this one, from all CTAs' thist ----
     const uint32_t th = smem_addr(thist);
     for (int e = tid; e < E; e += LC_THREADS) {
+        int v[LC_MAX_CTAS];
+#pragma unroll
+        for (int c = 0; c < LC_MAX_CTAS; ++c)  // independent remote loads, all in flight
+            v[c] = c < C ? ld_cluster_s32(cluster_map(th + 4u * e, (uint32_t)c)) : 0;
         int all = 0, below = 0;
-        for (int c = 0; c < C; ++c) {
-            const int v = ld_cluster_s32(cluster_map(th + 4u * e, (uint32_t)c));
-            all += v;
-            below += (uint32_t)c < me ? v : 0;
+#pragma unroll
+        for (int c = 0; c < LC_MAX_CTAS; ++c) {
+            all += v[c];
+            below += (uint32_t)c < me ? v[c] : 0;
         }
         s_tot[e] = all;
         s_base[e] = below;
     }
-    cluster_arrive();  // done reading the others' shared memory (waited for before exit)
+    cluster_arrive_relaxed();  // done reading the others' shared memory (waited for before exit)
     __syncthreads();
 
     // ---- exclusive scan of the padded counts over experts (one expert per thread) ----
@@ -764,10 +787,12 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
     bool launched = false;
+#ifndef MOE_NO_CLUSTER_LAYOUT
     cudaError_t ce = launch_layout_cluster(topk_idx, npairs, E, R, P, cap, counts, offsets, rank_offsets, slot_of,
                                            row_src, status, st, &launched);
     if (ce != cudaSuccess) return ce;
     if (launched) return cudaSuccess;
+#endif
     cudaError_t fe = launch_layout_fused(topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts, offsets,
                                          rank_offsets, slot_of, row_src, status, st, &launched);
     if (fe != cudaSuccess) return fe;

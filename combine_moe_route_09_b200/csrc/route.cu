@@ -184,9 +184,13 @@ __global__ void __launch_bounds__(SG_WARPS * 32)
         if (n_group > 1) {
             float a1 = NEG_INF, a2 = NEG_INF;
             if (my_g < n_group) {
+                // each group starts its scan at a different offset, so the lanes of
+                // one step read distinct banks (order does not change a top-2)
                 const float *grp = cs + my_g * gsize;
+                const int shift = (my_g * lpg) % gsize;
                 for (int i = my_sub; i < gsize; i += lpg) {
-                    const float v = grp[i];
+                    const int j = i + shift < gsize ? i + shift : i + shift - gsize;
+                    const float v = grp[j];
                     a2 = fmaxf(a2, fminf(a1, v));
                     a1 = fmaxf(a1, v);
                 }

@@ -142,6 +142,10 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 // Whole-CTA cluster barrier halves: every thread of every CTA of the cluster
 // arrives (release) and waits (acquire), from convergent code.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+// Arrival without release semantics: for a CTA that only signals "done reading".
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 // The shared::cluster address of `saddr` (a shared::cta address) in CTA `rank`.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
@@ -151,7 +155,7 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
 }
 __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
     int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 

@@ -16,6 +16,7 @@
  *   oracle_combine_fp8  the combine over e4m3 expert outputs with block scales
  *   oracle_route_sigmoid_grouped   router variant: sigmoid scores, selection-only
  *                       bias, group-limited top-K (with its exp / sigmoid)
+ *   oracle_route_weights_dispatched   routing weights in dispatched row order
  *   oracle_combine_backward / oracle_dispatch_backward / oracle_route_backward
  *                       the transposes of the steps (training)
  *   oracle_e4m3_encode / oracle_e4m3_decode / oracle_bf16_round   format helpers
