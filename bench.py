@@ -406,7 +406,7 @@ def run_ours(args, w, rank, world, local_rank):
         "dispatch_combine": {"tokens_per_s": w.S * world / (dc_ms * 1e-3), "effective_gb_s": dc_gbs,
                              "frac_of_peak": dc_gbs / peak, "frac_of_nominal_8tbs": dc_gbs / 8000.0},
         "phases": phases, "roofline": roofline, "e2e": e2e,
-        "gpu_launches": K * buf.KERNELS_PER_STEP, "clocks": clocks,
+        "gpu_launches": K * buf.kernels_per_step, "clocks": clocks,
         "timing": "value: K steps back to back (events at the ends only)"
                   + (", each step one CUDA-graph replay" if graph is not None else ", eager calls")
                   + "; phases/roofline: a second pass of K eager steps with an event between kernels",

@@ -31,6 +31,7 @@ from .binding import (  # noqa: F401
     moe_dispatch,
     moe_dispatch_backward,
     moe_dispatch_layout,
+    moe_dispatch_layout_kernels,
     moe_dispatch_layout_workspace,
     moe_dispatch_route_weights,
     moe_route_topk,

@@ -29,6 +29,7 @@ _P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 # name -> (restype, argtypes), the exact C signatures
 SIGNATURES = {
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_dispatch_layout_kernels": (_I, [_I, _I, _I]),
     "moe_dispatch_route_weights": (_I, [_P, _P, _I, _I, _L, _P, _P, _P]),
     "moe_route_sigmoid_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
@@ -120,6 +121,14 @@ def moe_route_topk(logits: torch.Tensor, K: int, topk_idx=None, topk_w=None, str
     _check("moe_route_topk", lib().moe_route_topk(_ptr(logits), S, E, K, _ptr(topk_idx), _ptr(topk_w),
                                                    _stream(stream, logits.device)))
     return topk_idx, topk_w
+
+
+def moe_dispatch_layout_kernels(S: int, E: int, K: int) -> int:
+    """Kernels moe_dispatch_layout launches for these sizes on the current device (1 or 2)."""
+    n = lib().moe_dispatch_layout_kernels(S, E, K)
+    if n < 0:
+        raise MoeError("moe_dispatch_layout_kernels", MOE_ERR_CUDA)
+    return n
 
 
 def moe_dispatch_route_weights(topk_w: torch.Tensor, row_src: torch.Tensor, out=None, status=None, stream=None):

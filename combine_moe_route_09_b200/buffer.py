@@ -31,9 +31,6 @@ class MoeBuffer:
     or bfloat16); fp8 = dispatch quantised to e4m3 with 128-channel scales.
     """
 
-    # kernels one step launches (route 1, layout 2, dispatch 1, combine 1)
-    KERNELS_PER_STEP = 5
-
     def __init__(self, S: int, H: int, K: int, E: int, R: int = 1, token_padding: int = 0,
                  dtype: torch.dtype = torch.bfloat16, fp8: bool = False, device="cuda"):
         if dtype not in (torch.float32, torch.bfloat16):
@@ -76,6 +73,12 @@ class MoeBuffer:
         self._p_slot, self._p_xd = p(L.slot_of), p(self.xd)
         self._p_xs = p(self.xs) if fp8 else None
         self._p_out, self._p_rnr = p(self.out), p(self.out_no_routed)
+
+    @property
+    def kernels_per_step(self) -> int:
+        """Kernels one step launches: route 1, layout 1 or 2, dispatch 1, combine 1."""
+        with torch.cuda.device(self.device):
+            return 3 + B.moe_dispatch_layout_kernels(self.S, self.E, self.K)
 
     @property
     def quant(self) -> int:

@@ -57,6 +57,11 @@ int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, 
                                         static_cast<cudaStream_t>(stream), current_sms()));
 }
 
+int moe_dispatch_layout_kernels(int S, int E, int K) {
+    if (S < 1 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK || (int64_t)S * K >= ((int64_t)1 << 31)) return 0;
+    return moe::layout_kernel_count(S, E, K);
+}
+
 int moe_dispatch_route_weights(const float *topk_w, const int32_t *row_src, int S, int K, int64_t cap,
                                float *route_weights, int32_t *status, void *stream) {
     if (S < 0 || K < 1 || K > MOE_MAX_TOPK || cap < 0 || cap >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;

@@ -56,6 +56,9 @@ cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias,
                                          int topk_group, int normalize, float scale, int32_t *idx, float *w,
                                          cudaStream_t st, int sms);
 
+// Kernels moe_dispatch_layout launches for these sizes on the current device (1 or 2; -1: CUDA error).
+int layout_kernel_count(int S, int E, int K);
+
 cudaError_t launch_route_weights(const float *topk_w, const int32_t *row_src, int64_t pairs, int64_t cap,
                                  float *out, int32_t *status, cudaStream_t st, int sms);
 

@@ -693,7 +693,7 @@ __global__ void __launch_bounds__(LC_THREADS)
 static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap,
                                          int32_t *counts, int32_t *offsets, int32_t *rank_offsets,
                                          int32_t *slot_of, int32_t *row_src, int32_t *status, cudaStream_t st,
-                                         bool *launched) {
+                                         bool *launched, bool dry = false) {
     *launched = false;
     const int C = (npairs + LC_TILE - 1) / LC_TILE;
     if (C < 1 || C > LC_MAX_CTAS) return cudaSuccess;  // not launched
@@ -705,6 +705,10 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     if (per_sm < 1) return cudaSuccess;
     static int pdl_ok = 1, cluster_ok = 1;
     if (!cluster_ok) return cudaSuccess;
+    if (dry) {
+        *launched = true;
+        return cudaSuccess;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C);
     cfg.blockDim = dim3(LC_THREADS);
@@ -740,7 +744,7 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
 static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap, int T,
                                        int32_t *hist, LayoutHeader *hdr, int32_t *counts, int32_t *offsets,
                                        int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src, int32_t *status,
-                                       cudaStream_t st, bool *launched) {
+                                       cudaStream_t st, bool *launched, bool dry = false) {
     *launched = false;
     const size_t smem = (size_t)((LT_WARPS * E * 2 + 15) & ~15) + 2 * 1024 * sizeof(int);
     static KernelSlots<decltype(&layout_fused_kernel)> slots;
@@ -750,6 +754,10 @@ static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int 
     long long grid = (long long)sms * per_sm;  // all CTAs must be co-resident
     if (grid > T) grid = T;
     if (grid < 1 || (long long)T * E > LF_MAX_HIST) return cudaSuccess;  // not launched: use two kernels
+    if (dry) {
+        *launched = true;
+        return cudaSuccess;
+    }
     // Cooperative (all CTAs co-resident, for the grid barrier) and, where the
     // driver accepts the pair, programmatic serialisation too (see pdl_wait).
     static int pdl_ok = 1;
@@ -776,6 +784,21 @@ static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int 
     }
     if (e == cudaSuccess) *launched = true;
     return e;
+}
+
+int layout_kernel_count(int S, int E, int K) {
+    const int npairs = S * K;
+    bool one = false;
+#ifndef MOE_NO_CLUSTER_LAYOUT
+    if (launch_layout_cluster(nullptr, npairs, E, 1, 0, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                              nullptr, &one, true) != cudaSuccess)
+        return -1;
+    if (one) return 1;
+#endif
+    if (launch_layout_fused(nullptr, npairs, E, 1, 0, 0, layout_tiles(npairs), nullptr, nullptr, nullptr, nullptr,
+                            nullptr, nullptr, nullptr, nullptr, nullptr, &one, true) != cudaSuccess)
+        return -1;
+    return one ? 1 : 2;
 }
 
 cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int P,

@@ -162,8 +162,16 @@ __global__ void __launch_bounds__(SG_WARPS * 32)
     while (lpg * 2 * n_group <= 32) lpg *= 2;
     const int my_g = lane / lpg, my_sub = lane - my_g * lpg;
     const float NEG_INF = __int_as_float(0xff800000);
+    // group of expert e (< 1024) = umulhi(e, ceil(2^32 / gsize)), exact for gsize >= 2
+    const uint32_t gmagic = n_group > 1 ? 0xffffffffu / (uint32_t)gsize + 1u : 0u;
+    float bv[NPER];
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) bv[j] = (bias && lane + 32 * j < E) ? __ldg(bias + lane + 32 * j) : 0.f;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
         const float *row = logits + (size_t)t * E;
+        float lv[NPER];
+#pragma unroll
+        for (int j = 0; j < NPER; ++j) lv[j] = lane + 32 * j < E ? __ldg(row + lane + 32 * j) : 0.f;
         float cv[NPER];
 #pragma unroll
         for (int j = 0; j < NPER; ++j) {
@@ -172,8 +180,8 @@ __global__ void __launch_bounds__(SG_WARPS * 32)
             if (e < E) {
                 // sigmoid = 1 / (1 + exp(-l)): the correctly rounded reciprocal is the
                 // correctly rounded quotient 1 / d
-                const float sg = __frcp_rn(__fadd_rn(1.0f, route_exp(-__ldg(row + e))));
-                cv[j] = bias ? __fadd_rn(sg, __ldg(bias + e)) : sg;
+                const float sg = __frcp_rn(__fadd_rn(1.0f, route_exp(-lv[j])));
+                cv[j] = bias ? __fadd_rn(sg, bv[j]) : sg;
                 cs[e] = cv[j];
                 ss[e] = sg;
             }
@@ -220,7 +228,7 @@ __global__ void __launch_bounds__(SG_WARPS * 32)
         for (int j = 0; j < NPER; ++j) {
             const int e = lane + 32 * j;
             bool ok = e < E;
-            if (n_group > 1 && ok) ok = (keep >> ((e / gsize) * lpg)) & 1u;
+            if (n_group > 1 && ok) ok = (keep >> (__umulhi((uint32_t)e, gmagic) * lpg)) & 1u;
             key[j] = ok ? ordered_bits(cv[j]) : 0u;
         }
         int my_e = 0;

@@ -109,6 +109,16 @@ MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *to
                    void *stream);
 
 /*
+ * Number of kernels moe_dispatch_layout (and moe_dispatch_layout_static)
+ * launches for these sizes on the current device: 1 (single-launch layouts:
+ * a thread-block cluster for up to 32768 pairs, else a cooperative grid when
+ * every CTA can scan the tile histograms) or 2 (histogram + slots).  For
+ * sizing CUDA graphs and counting launches; no launch happens.  Returns -1 on
+ * a CUDA error, 0 for invalid sizes.
+ */
+MOE_API int moe_dispatch_layout_kernels(int S, int E, int K);
+
+/*
  * Routing weights in dispatched order (MoonEP developer guide, core API
  * example: the dispatch returns each expert's rows together with their routing
  * weights, which the combine consumes).

@@ -304,6 +304,16 @@ def test_layout_paths_large(S, E, K, R, P):
     assert status.item() == 0
 
 
+@pytest.mark.parametrize("S,E,K,n", [
+    (4096, 256, 8, 1),       # cluster layout
+    (1, 7, 2, 1),
+    (150000, 64, 8, 1),      # cooperative single launch
+    (8192, 1024, 32, 2),     # histogram + slots
+])
+def test_layout_kernel_count(S, E, K, n):
+    assert B.moe_dispatch_layout_kernels(S, E, K) == n
+
+
 def test_kernels_accept_any_size_order():
     """Launch shapes whose shared-memory needs go up, down and up again."""
     rng = np.random.default_rng(9)
