@@ -514,11 +514,17 @@ __global__ void __launch_bounds__(LT_THREADS)
 // shared memory alive until the others have read it.
 // ------------------------------------------------------------------------------------------
 
-constexpr int LC_WARPS = 32;
+#ifndef MOE_LC_WARPS
+#define MOE_LC_WARPS 32
+#endif
+#ifndef MOE_LC_MAX_CTAS
+#define MOE_LC_MAX_CTAS 8
+#endif
+constexpr int LC_WARPS = MOE_LC_WARPS;
 constexpr int LC_THREADS = LC_WARPS * 32;
 constexpr int LC_ITEMS = 4;
-constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // 4096 pairs
-constexpr int LC_MAX_CTAS = 8;                 // portable cluster size
+constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // pairs per CTA (4096 with 32 warps)
+constexpr int LC_MAX_CTAS = MOE_LC_MAX_CTAS;   // 8: the portable cluster size
 
 __global__ void __launch_bounds__(LC_THREADS)
     layout_cluster_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P, int64_t cap,
@@ -530,14 +536,16 @@ __global__ void __launch_bounds__(LC_THREADS)
     int *s_tot = thist + E;                                     // [E] totals
     int *s_base = s_tot + E;                                    // [E] first row of this tile's pairs, per expert
     int *s_off = s_base + E;                                    // [E + 1] padded offsets
-    uint16_t *whist = reinterpret_cast<uint16_t *>(s_off + E + 1 + 3);  // [LC_WARPS][E]
+    // [LC_WARPS][E + 2]: the padded row stride moves each warp's row by one bank
+    uint16_t *whist = reinterpret_cast<uint16_t *>(s_off + E + 1 + 3);
+    const int WS = E + 2;
     __shared__ int s_wsum[LC_WARPS];
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int C = gridDim.x;
     const uint32_t me = cluster_ctarank();
     const int tile = blockIdx.x;
-    for (int i = tid; i < LC_WARPS * E; i += LC_THREADS) whist[i] = 0;
+    for (int i = tid; i < LC_WARPS * WS; i += LC_THREADS) whist[i] = 0;
     __syncthreads();
     pdl_wait();
     pdl_trigger();
@@ -561,9 +569,9 @@ __global__ void __launch_bounds__(LC_THREADS)
             e = -1;
         }
         const unsigned peers = __match_any_sync(FULL, e);
-        const int before = e >= 0 ? (int)whist[w * E + e] : 0;
+        const int before = e >= 0 ? (int)whist[w * WS + e] : 0;
         __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
+        if (e >= 0 && lane == __ffs(peers) - 1) whist[w * WS + e] = (uint16_t)(before + __popc(peers));
         __syncwarp();
         my_e[it] = e;
         my_r[it] = before + __popc(peers & lt);
@@ -574,7 +582,7 @@ __global__ void __launch_bounds__(LC_THREADS)
     // expert: tpe consecutive lanes share an expert, each summing LC_WARPS / tpe
     // warps, then an exclusive scan across those lanes (shuffles)
     int tpe = 1;
-    while (tpe < 32 && tpe * 2 * E <= LC_THREADS) tpe *= 2;
+    while (tpe < 32 && tpe < LC_WARPS && tpe * 2 * E <= LC_THREADS) tpe *= 2;
     {
         const int wpt = LC_WARPS / tpe, sub = lane & (tpe - 1), epw = 32 / tpe;
         const int w0 = sub * wpt;
@@ -583,7 +591,7 @@ __global__ void __launch_bounds__(LC_THREADS)
             const bool ok = e < E;
             int part = 0;
             if (ok)
-                for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * E + e];
+                for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * WS + e];
             int incl = part;  // inclusive scan over the tpe lanes of this expert
             for (int off = 1; off < tpe; off <<= 1) {
                 const int o = __shfl_up_sync(FULL, incl, off, tpe);
@@ -592,8 +600,8 @@ __global__ void __launch_bounds__(LC_THREADS)
             if (ok) {
                 int run = incl - part;
                 for (int ww = w0; ww < w0 + wpt; ++ww) {
-                    const int c = whist[ww * E + e];
-                    whist[ww * E + e] = (uint16_t)run;
+                    const int c = whist[ww * WS + e];
+                    whist[ww * WS + e] = (uint16_t)run;
                     run += c;
                 }
                 if (sub == tpe - 1) thist[e] = incl;
@@ -633,13 +641,13 @@ __global__ void __launch_bounds__(LC_THREADS)
     if (lane == 31) s_wsum[w] = incl;
     __syncthreads();
     if (w == 0) {
-        int v = s_wsum[lane];
+        int v = lane < LC_WARPS ? s_wsum[lane] : 0;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(FULL, v, off);
             if (lane >= off) v += o;
         }
-        s_wsum[lane] = v;  // inclusive over warps
+        if (lane < LC_WARPS) s_wsum[lane] = v;  // inclusive over warps
     }
     __syncthreads();
     if (tid < E) {
@@ -666,7 +674,7 @@ __global__ void __launch_bounds__(LC_THREADS)
         const int e = my_e[it];
         int sl = -1;
         if (e >= 0) {
-            sl = s_base[e] + whist[w * E + e] + my_r[it];
+            sl = s_base[e] + whist[w * WS + e] + my_r[it];
             if ((int64_t)sl >= cap) {
                 sl = -1;
                 over = true;
@@ -696,8 +704,8 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
                                          bool *launched, bool dry = false) {
     *launched = false;
     const int C = (npairs + LC_TILE - 1) / LC_TILE;
-    if (C < 1 || C > LC_MAX_CTAS) return cudaSuccess;  // not launched
-    const size_t smem = (size_t)(4 * E + 4) * sizeof(int) + (size_t)LC_WARPS * E * sizeof(uint16_t);
+    if (C < 1 || C > LC_MAX_CTAS || E > LC_THREADS) return cudaSuccess;  // not launched
+    const size_t smem = (size_t)(4 * E + 4) * sizeof(int) + (size_t)LC_WARPS * (E + 2) * sizeof(uint16_t);
     static KernelSlots<decltype(&layout_cluster_kernel)> slots;
     int sms = 0, per_sm = 0;
     cudaError_t e = slots.prepare(&layout_cluster_kernel, LC_THREADS, smem, &sms, &per_sm);
@@ -708,6 +716,14 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     if (dry) {
         *launched = true;
         return cudaSuccess;
+    }
+    if (C > 8) {  // clusters above the portable size must be allowed per function
+        e = cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            cluster_ok = 0;
+            return cudaSuccess;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C);
