@@ -505,8 +505,8 @@ __global__ void __launch_bounds__(LT_THREADS)
 
 // ------------------------------------------------------------------------------------------
 // Cluster layout: up to LC_MAX_CTAS tiles of LC_TILE pairs, one CTA each, all
-// in one thread-block cluster.  Each CTA ranks its tile (as above, with 32
-// warps), keeps the tile histogram in its own shared memory, and after one
+// in one thread-block cluster (E <= LC_THREADS).  Each CTA ranks its tile (as
+// above), keeps the tile histogram in its own shared memory, and after one
 // hardware cluster barrier reads the other CTAs' histograms through
 // distributed shared memory: the per-expert totals and the counts of the tiles
 // below it.  No global scratch, no atomics, no spin-wait.  A second cluster
@@ -515,16 +515,19 @@ __global__ void __launch_bounds__(LT_THREADS)
 // ------------------------------------------------------------------------------------------
 
 #ifndef MOE_LC_WARPS
-#define MOE_LC_WARPS 32
+#define MOE_LC_WARPS 16
 #endif
 #ifndef MOE_LC_MAX_CTAS
-#define MOE_LC_MAX_CTAS 8
+#define MOE_LC_MAX_CTAS 16
 #endif
 constexpr int LC_WARPS = MOE_LC_WARPS;
 constexpr int LC_THREADS = LC_WARPS * 32;
 constexpr int LC_ITEMS = 4;
-constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // pairs per CTA (4096 with 32 warps)
-constexpr int LC_MAX_CTAS = MOE_LC_MAX_CTAS;   // 8: the portable cluster size
+constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // 2048 pairs per CTA
+// 16 CTAs: above the portable cluster size of 8, allowed per function (the
+// layout falls back to the other paths where the device refuses it).  In the
+// DeepSeek-V3-shaped prefill step, 16 CTAs of 512 threads beat 8 CTAs of 1024.
+constexpr int LC_MAX_CTAS = MOE_LC_MAX_CTAS;
 
 __global__ void __launch_bounds__(LC_THREADS)
     layout_cluster_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P, int64_t cap,

@@ -111,7 +111,7 @@ MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *to
 /*
  * Number of kernels moe_dispatch_layout (and moe_dispatch_layout_static)
  * launches for these sizes on the current device: 1 (single-launch layouts:
- * a thread-block cluster for up to 32768 pairs, else a cooperative grid when
+ * a thread-block cluster for up to 32768 pairs and E <= 512, else a cooperative grid when
  * every CTA can scan the tile histograms) or 2 (histogram + slots).  For
  * sizing CUDA graphs and counting launches; no launch happens.  Returns -1 on
  * a CUDA error, 0 for invalid sizes.

@@ -285,8 +285,10 @@ def test_fp8_quotients_near_rounding_midpoints(in_bf16):
     (8192, 1024, 32, 8, 16),   # T*E above the fused layout's scan bound: the two-kernel layout
     (150000, 64, 8, 8, 128),   # more tiles than co-resident CTAs: several tiles per CTA (fused)
     (20000, 512, 8, 4, 0),     # mid-size fused
-    (1024, 1024, 32, 8, 16),   # cluster layout: 8 CTAs of 4096 pairs, the largest E
+    (1024, 512, 32, 8, 16),    # cluster layout: 16 CTAs of 2048 pairs, the largest E it takes
+    (1024, 1024, 32, 8, 16),   # the same pairs with E = 1024: cooperative single launch
     (4095, 256, 8, 8, 0),      # cluster layout, ragged last tile
+    (1000, 300, 8, 3, 0),      # cluster of 4 CTAs, E not a multiple of 32
     (4097, 256, 8, 8, 128),    # one tile past the cluster layout's bound: fused
     (3, 7, 2, 1, 5),           # cluster of one CTA, E not a multiple of 32
 ])
@@ -307,6 +309,7 @@ def test_layout_paths_large(S, E, K, R, P):
 @pytest.mark.parametrize("S,E,K,n", [
     (4096, 256, 8, 1),       # cluster layout
     (1, 7, 2, 1),
+    (1024, 1024, 32, 1),     # E above the cluster layout's bound: cooperative
     (150000, 64, 8, 1),      # cooperative single launch
     (8192, 1024, 32, 2),     # histogram + slots
 ])
