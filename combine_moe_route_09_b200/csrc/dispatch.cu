@@ -157,6 +157,10 @@ constexpr int DQ_UNITS = 2;                                  // units per thread
 constexpr int DQ_SPAN = DQ_CONSUMERS * DQ_UNIT;              // channels between a thread's units
 constexpr int DQ_MAX_BLOCKS = DQ_UNITS * DQ_SPAN / 128;      // 128-channel blocks per item
 constexpr int DQ_HDR = 128;                                  // per-stage header: the token's K slots
+#ifndef MOE_DQ_BULK
+#define MOE_DQ_BULK 1
+#endif
+constexpr int DQ_OUT_BUFS = 2;                               // bulk-store path: output staging buffers
 
 struct Fp8Args {
     const uint8_t *x;
@@ -171,6 +175,8 @@ struct Fp8Args {
     int nchunks;     // items per token
     int stage;       // bytes per stage: header + bpc * 128 * esz
     int stages;      // stages in the ring (<= DQ_MAX_STAGES)
+    int obuf;        // bulk-store path: bytes per output staging buffer (codes, then scales)
+    int scale_bulk;  // bulk-store path: the item's scale segment is also one bulk store per copy
 };
 
 // s = amax / 448 rounded to nearest even.  For amax >= 2^-80 this is
@@ -235,15 +241,19 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
     return U4{w[0], w[1], w[2], w[3]};
 }
 
-// KT: K known at compile time (0 = runtime K).
-template <bool IN_F32, int KT>
+// KT: K known at compile time (0 = runtime K).  BULK: the K copies of an item
+// leave through TMA bulk stores from a shared-memory staging buffer (one
+// elected thread issues them) instead of per-thread 16-byte stores.
+template <bool IN_F32, int KT, bool BULK>
 __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kernel(const Fp8Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    // layout: [stages][header (K slots) | bpc*128*esz input bytes] | barriers
+    // layout: [stages][header (K slots) | bpc*128*esz input bytes]
+    //         | BULK: [DQ_OUT_BUFS][bpc*128 codes | bpc*4 scales, padded to 16] | barriers
     const int NS = a.stages;
     const int K = KT > 0 ? KT : a.K;
     const uint32_t smem0 = smem_addr(smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * a.stage);
+    const uint32_t obuf0 = smem0 + (uint32_t)(NS * a.stage);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * a.stage + (BULK ? DQ_OUT_BUFS * a.obuf : 0));
     const uint32_t bar0 = smem_addr(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (DQ_MAX_STAGES + s); };
@@ -318,7 +328,16 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
     int i = 0;
     for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
         const int s = i % NS;
-        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / NS) & 1, a.status))) break;
+        if constexpr (BULK) {
+            // All 128 consumers leave together on a timeout (the staging buffer and
+            // the barriers below are shared); the issuing thread first lets the
+            // stores that last read this item's staging buffer finish reading it.
+            const bool got = mbar_wait(full_bar(s), (i / NS) & 1, a.status);
+            if (tid == 0) bulk_wait_read<DQ_OUT_BUFS - 1>();
+            if (!named_bar_and(1, DQ_CONSUMERS, got)) break;
+        } else {
+            if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / NS) & 1, a.status))) break;
+        }
         const int col0 = c * a.bpc * 128;              // first channel of the item
         const int nch = min(a.bpc * 128, a.H - col0);  // channels in this item
         const uint32_t st = smem0 + (uint32_t)(s * a.stage);
@@ -380,6 +399,45 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
         }
 
         const bool lead = (lane & 7) == 0;
+        if constexpr (BULK) {
+            // stage the item (codes, then its scales), then one thread sends K copies
+            const uint32_t ob = obuf0 + (uint32_t)((i % DQ_OUT_BUFS) * a.obuf);
+            const int cbytes = a.bpc * 128;
+#pragma unroll
+            for (int u = 0; u < DQ_UNITS; ++u) {
+                if (active[u]) {
+                    const int ch = u * DQ_SPAN + tid * DQ_UNIT;
+                    sts128(ob + (uint32_t)ch, q[u]);
+                    if (lead) asm volatile("st.shared.f32 [%0], %1;" ::"r"(ob + (uint32_t)(cbytes + (ch >> 7) * 4)),
+                                           "f"(scale[u]) : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar(2, DQ_CONSUMERS);
+            const int nblk = nch >> 7;
+            if (warp == 0) {
+                for (int k = 0; k < K; ++k) {
+                    const int sl = __shfl_sync(FULL, myslot, k);
+                    if (lane == 0 && sl >= 0) {
+                        bulk_s2g(a.xd + (size_t)sl * a.H + col0, ob, (uint32_t)nch);
+                        if (a.scale_bulk)
+                            bulk_s2g(a.xs + (size_t)sl * nb + (col0 >> 7), ob + (uint32_t)cbytes, (uint32_t)nblk * 4u);
+                    }
+                }
+                if (lane == 0) bulk_commit();
+            }
+            if (!a.scale_bulk) {  // scales from registers, by each block's lead thread
+                float *const scol = a.xs + ((col0 + tid * DQ_UNIT) >> 7);
+                for (int k = 0; k < K; ++k) {
+                    const int sl = __shfl_sync(FULL, myslot, k);
+                    if (sl < 0 || !lead) continue;
+#pragma unroll
+                    for (int u = 0; u < DQ_UNITS; ++u)
+                        if (active[u]) scol[(size_t)sl * nb + u * (DQ_SPAN >> 7)] = scale[u];
+                }
+            }
+            continue;
+        }
         uint8_t *const xcol = a.xd + col0 + tid * DQ_UNIT;
         float *const scol = a.xs + ((col0 + tid * DQ_UNIT) >> 7);
         constexpr int KU = KT > 0 ? KT : 1;
@@ -397,6 +455,9 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
                 }
             }
         }
+    }
+    if constexpr (BULK) {
+        if (tid == 0) bulk_wait_all();  // this CTA's bulk stores are complete before it exits
     }
 }
 
@@ -434,16 +495,21 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
     }
     Fp8Args a{reinterpret_cast<const uint8_t *>(x), slot_of, reinterpret_cast<uint8_t *>(xd), xs, status,
               cap, S, H, K, esz, 0, 0, 0, 0};
-    // Split each row into the fewest items of at most DQ_MAX_BLOCKS blocks, as evenly as possible.
+    // Split each row into the fewest items of at most DQ_MAX_BLOCKS blocks, as evenly as possible
+    // (a multiple of 4 blocks where the row allows, so scale segments are whole 16-byte units).
     const int blocks = H / 128;
     const int n = (blocks + DQ_MAX_BLOCKS - 1) / DQ_MAX_BLOCKS;
     a.bpc = (blocks + n - 1) / n;
+    if (blocks % 4 == 0) a.bpc = (a.bpc + 3) / 4 * 4;
     a.nchunks = (blocks + a.bpc - 1) / a.bpc;
     a.stage = DQ_HDR + a.bpc * 128 * esz;
     a.stages = DQ_STAGE_BUDGET / a.stage;
     if (a.stages > DQ_MAX_STAGES) a.stages = DQ_MAX_STAGES;
     if (a.stages < 3) a.stages = 3;
-    const size_t smem = (size_t)a.stages * a.stage + 2 * DQ_MAX_STAGES * 8;
+    a.obuf = a.bpc * 128 + (a.bpc * 4 + 15) / 16 * 16;
+    a.scale_bulk = (blocks % 4 == 0 && a.bpc % 4 == 0 && (reinterpret_cast<uintptr_t>(xs) & 15) == 0) ? 1 : 0;
+    const bool bulk = MOE_DQ_BULK != 0;
+    const size_t smem = (size_t)a.stages * a.stage + (bulk ? (size_t)DQ_OUT_BUFS * a.obuf : 0) + 2 * DQ_MAX_STAGES * 8;
     const long long nitems = (long long)S * a.nchunks;
     auto go = [&](auto kern) -> cudaError_t {
         static KernelSlots<decltype(kern)> slots;
@@ -452,9 +518,10 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3(grid), dim3(DQ_THREADS), smem, st, a);
     };
+    constexpr bool BK = MOE_DQ_BULK != 0;
     if (dtype == MOE_DTYPE_BF16)
-        return K == 8 ? go(&dispatch_fp8_kernel<false, 8>) : go(&dispatch_fp8_kernel<false, 0>);
-    return K == 8 ? go(&dispatch_fp8_kernel<true, 8>) : go(&dispatch_fp8_kernel<true, 0>);
+        return K == 8 ? go(&dispatch_fp8_kernel<false, 8, BK>) : go(&dispatch_fp8_kernel<false, 0, BK>);
+    return K == 8 ? go(&dispatch_fp8_kernel<true, 8, BK>) : go(&dispatch_fp8_kernel<true, 0, BK>);
 }
 
 }  // namespace moe

@@ -269,6 +269,43 @@ def _midpoint_blocks(rng, S, H, in_bf16: bool):
     return synth.f32_to_bf16_bits(x) if in_bf16 else x
 
 
+@pytest.mark.parametrize("H,K", [(640, 8), (1664, 3), (4224, 8), (7296, 8), (7168, 5), (512, 32)])
+def test_fp8_dispatch_row_shapes(H, K):
+    """Rows whose block count is or is not a multiple of 4 (scale segments sent as one
+    bulk store per copy, or stored per block), one or two items per row, small and large K;
+    slots scattered over a larger capacity with unused rows left untouched."""
+    rng = np.random.default_rng(H + K)
+    S = 300
+    cap = S * K + 77
+    x = synth.f32_to_bf16_bits((rng.standard_normal((S, H)) * rng.uniform(0.01, 50, (S, 1))).astype(np.float32))
+    slot = rng.permutation(cap)[:S * K].astype(np.int32).reshape(S, K)
+    ref_xd, ref_xs = oracle.dispatch(x, slot, cap, quant=oracle.QUANT_FP8_E4M3_B128)
+    xd = torch.full((cap, H), 0x5A, dtype=torch.uint8, device="cuda").view(torch.float8_e4m3fn)
+    xs = torch.full((cap, H // 128), -7.0, dtype=torch.float32, device="cuda")
+    B.moe_dispatch(dev(x), dev(slot), cap, B.MOE_QUANT_FP8_E4M3_B128, xd=xd, xs=xs)
+    used = np.zeros(cap, bool)
+    used[slot.reshape(-1)] = True
+    np.testing.assert_array_equal(host(xd)[used], ref_xd[used])
+    np.testing.assert_array_equal(host(xs)[used], ref_xs[used])
+    assert np.all(host(xd.view(torch.uint8))[~used] == 0x5A) and np.all(host(xs)[~used] == -7.0)
+
+
+def test_fp8_dispatch_scale_rows_not_16_byte_aligned():
+    """A scale array whose base is only 4-byte aligned: scales are stored per block."""
+    rng = np.random.default_rng(5)
+    S, H, K = 64, 2048, 4
+    cap = S * K
+    x = synth.f32_to_bf16_bits(rng.standard_normal((S, H)).astype(np.float32))
+    slot = rng.permutation(cap).astype(np.int32).reshape(S, K)
+    ref_xd, ref_xs = oracle.dispatch(x, slot, cap, quant=oracle.QUANT_FP8_E4M3_B128)
+    big = torch.zeros(cap * (H // 128) + 1, dtype=torch.float32, device="cuda")
+    xs = big[1:].view(cap, H // 128)  # base + 4 bytes
+    xd = torch.empty((cap, H), dtype=torch.float8_e4m3fn, device="cuda")
+    B.moe_dispatch(dev(x), dev(slot), cap, B.MOE_QUANT_FP8_E4M3_B128, xd=xd, xs=xs)
+    np.testing.assert_array_equal(host(xd), ref_xd)
+    np.testing.assert_array_equal(host(xs), ref_xs)
+
+
 @pytest.mark.parametrize("in_bf16", [False, True])
 def test_fp8_quotients_near_rounding_midpoints(in_bf16):
     rng = np.random.default_rng(8 + in_bf16)
