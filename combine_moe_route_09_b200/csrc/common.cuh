@@ -1,6 +1,8 @@
 // Shared device helpers of the sm_100a MoE routing kernels.
 #pragma once
 
+#include <mutex>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -94,47 +96,66 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// Per-kernel launch facts, computed once per (device, dynamic shared memory
-// size): how many CTAs of that size fit on one SM.  The kernel's opt-in limit
-// for dynamic shared memory is one setting per device that the last call
-// wins, so it is only ever raised, to the largest size requested so far, and
-// every smaller launch stays within it.  A handful of sizes per kernel are
-// cached; beyond that the query simply runs again.  Races between host
-// threads only repeat idempotent driver calls.
+// Launch facts per (device, kernel, block size, dynamic shared memory size):
+// how many CTAs fit on one SM.  A kernel's opt-in limit for dynamic shared
+// memory is one setting per device and kernel that the last call wins, so it
+// is only ever raised, to the largest size requested so far, and every smaller
+// launch stays within it.  Up to 32 (device, kernel) pairs and 32 occupancy
+// answers are cached; beyond that the calls simply run again.  A mutex guards
+// the tables against concurrent host threads.
 template <typename Kern>
 struct KernelSlots {
-    static constexpr int N = 8;
-    static constexpr int MAXDEV = 64;
-    int dev[N] = {-1, -1, -1, -1, -1, -1, -1, -1};
-    size_t smem[N] = {};
-    int sms[N] = {}, per_sm[N] = {};
-    int next = 0;
-    size_t limit_set[MAXDEV] = {};
-    bool carveout_set[MAXDEV] = {};
+    // One object may serve several kernels of the same signature (template
+    // instances), so every cached fact is keyed by (device, kernel).
+    static constexpr int N = 32;
+    struct Attr {
+        int dev = -1;
+        Kern kern = nullptr;
+        size_t limit = 0;  // largest dynamic shared memory set so far (the attribute only grows)
+    };
+    struct Occ {
+        int dev = -1;
+        Kern kern = nullptr;
+        int threads = 0;
+        size_t smem = 0;
+        int sms = 0, per_sm = 0;
+    };
+    Attr attr[N];
+    Occ occ[N];
+    int n_attr = 0, next_occ = 0;
+    std::mutex mu;
 
     cudaError_t prepare(Kern kern, int threads, size_t bytes, int *n_sms, int *n_per_sm) {
         int d = 0;
         cudaError_t e = cudaGetDevice(&d);
         if (e != cudaSuccess) return e;
-        if (d < 0 || d >= MAXDEV) return cudaErrorInvalidDevice;
-        if (bytes > limit_set[d]) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-            if (e != cudaSuccess) return e;
-            limit_set[d] = bytes;
-        }
-        if (!carveout_set[d]) {
-            // Every kernel of the library asks for the largest shared-memory
-            // carveout, so consecutive kernels never wait for an L1/shared
-            // split to be reconfigured.
+        std::lock_guard<std::mutex> lock(mu);
+        Attr *a = nullptr;
+        for (int i = 0; i < n_attr; ++i)
+            if (attr[i].dev == d && attr[i].kern == kern) a = &attr[i];
+        if (!a) {
+            // First use on this device: ask for the largest shared-memory carveout,
+            // so consecutive kernels never wait for an L1/shared split to be
+            // reconfigured.
             e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
-            carveout_set[d] = true;
+            if (n_attr < N) {
+                a = &attr[n_attr++];
+                a->dev = d;
+                a->kern = kern;
+            }
+        }
+        if (!a || bytes > a->limit) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+            if (e != cudaSuccess) return e;
+            if (a) a->limit = bytes;
         }
         for (int i = 0; i < N; ++i) {
-            if (dev[i] == d && smem[i] == bytes) {
-                *n_sms = sms[i];
-                *n_per_sm = per_sm[i];
+            const Occ &o = occ[i];
+            if (o.dev == d && o.kern == kern && o.threads == threads && o.smem == bytes) {
+                *n_sms = o.sms;
+                *n_per_sm = o.per_sm;
                 return cudaSuccess;
             }
         }
@@ -144,11 +165,13 @@ struct KernelSlots {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p, kern, threads, bytes);
         if (e != cudaSuccess) return e;
         if (p < 1) p = 1;
-        const int i = next++ % N;
-        sms[i] = s;
-        per_sm[i] = p;
-        smem[i] = bytes;
-        dev[i] = d;
+        Occ &o = occ[next_occ++ % N];
+        o.dev = d;
+        o.kern = kern;
+        o.threads = threads;
+        o.smem = bytes;
+        o.sms = s;
+        o.per_sm = p;
         *n_sms = s;
         *n_per_sm = p;
         return cudaSuccess;
