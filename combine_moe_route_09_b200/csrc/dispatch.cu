@@ -25,9 +25,13 @@
 //    block reduce amax with xor-shuffles, s = amax / 448 (IEEE division) and
 //    q = e4m3(x / s) with the quotient correctly rounded (Markstein's
 //    correction of x * RN(1/s); plain IEEE division for subnormal s) and
-//    cvt.rn.satfinite.e4m3x2.  Each thread stores its 16 codes K times from
-//    registers (a warp writes 512 contiguous bytes per copy); the block's
-//    lead thread stores the scale.
+//    cvt.rn.satfinite.e4m3x2.  The quantised item (codes, then its block
+//    scales) is staged in one of DQ_OUT_BUFS shared-memory buffers, and after a named
+//    barrier one thread sends the K copies as TMA bulk stores (one per copy
+//    for the codes, one for the scales when the segment is whole 16-byte
+//    units, else the blocks' lead threads store the scales).  Whole-row bulk
+//    stores write the scattered destination rows faster than per-thread
+//    16-byte stores.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tma.cuh"
@@ -160,7 +164,10 @@ constexpr int DQ_HDR = 128;                                  // per-stage header
 #ifndef MOE_DQ_BULK
 #define MOE_DQ_BULK 1
 #endif
-constexpr int DQ_OUT_BUFS = 2;                               // bulk-store path: output staging buffers
+#ifndef MOE_DQ_OUT_BUFS
+#define MOE_DQ_OUT_BUFS 2
+#endif
+constexpr int DQ_OUT_BUFS = MOE_DQ_OUT_BUFS;                 // bulk-store path: output staging buffers
 
 struct Fp8Args {
     const uint8_t *x;
