@@ -12,10 +12,7 @@
 // Persistent kernel on the same pipeline as the forward combine: a producer
 // warp bulk-loads, per (token, chunk) item, the K gathered y chunks, the g
 // chunk and the gn chunk into a 4-stage ring (cp.async.bulk, mbarriers, no
-// multicast); 4 consumer warps hold one 16-byte unit per thread.  grad_y is
-// written back into the stage over the y chunks it replaces and leaves as K
-// bulk stores issued by one thread; a stage is freed one item later, once
-// those stores have read it.  Each CTA
+// multicast); 4 consumer warps hold one 16-byte unit per thread.  Each CTA
 // takes whole tokens, so grad_w needs no atomics: per item every warp reduces
 // its dot-product partials with a fixed xor tree and lane k keeps pair k's
 // running sum; at the token's last chunk the four warps' sums are added in
@@ -34,12 +31,6 @@ constexpr int BW_THREADS = BW_CONSUMERS + 32;
 constexpr int BW_MAX_CHUNK = BW_CONSUMERS * 16;
 constexpr int BW_HDR = 384;  // per stage: valid mask, the token's K weights (at 4), K slots (at 132)
 constexpr int BW_SMEM_BUDGET = 100 * 1024;
-#ifndef MOE_BW_BULK
-#define MOE_BW_BULK 1
-#endif
-// grad_y leaves through TMA bulk stores: each thread overwrites its unit of the
-// y_k chunk in the stage with w_k g, and one thread sends the K chunks.
-constexpr bool BW_BULK = MOE_BW_BULK != 0;
 
 struct CombineBwdArgs {
     const uint8_t *g, *gn, *y;
@@ -102,7 +93,7 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     if (tid == 0) {
         for (int s = 0; s < BW_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), BW_BULK ? 1 : BW_CONSUMER_WARPS);
+            mbar_init(empty_bar(s), BW_CONSUMER_WARPS);
         }
         fence_mbar_init();
     }
@@ -219,13 +210,9 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
                             p = __fmaf_rn(yf[e], gf[e], p);
                             gy[e] = __fmul_rn(wk, gf[e]);
                         }
-                        if constexpr (BW_BULK) {
-                            sts128(data + (uint32_t)(k * chunk + ub), V::pack(gy));
-                        } else {
-                            int sl;
-                            asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * k) : "memory");
-                            st_v4(a.grad_y + (size_t)sl * a.row_bytes + off + ub, V::pack(gy));
-                        }
+                        int sl;
+                        asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * k) : "memory");
+                        st_v4(a.grad_y + (size_t)sl * a.row_bytes + off + ub, V::pack(gy));
                     }
                     // fixed xor tree: every lane ends with the warp's partial for pair k
 #pragma unroll
@@ -233,33 +220,8 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
                     if (lane == k) run += p;
                 }
             }
-            if constexpr (!BW_BULK) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-            }
-        }
-        if constexpr (BW_BULK) {
-            // Every consumer is done with the stage (its reads, and its grad_y units
-            // written in place); one thread sends the K grad_y chunks, then frees
-            // the previous item's stage once that item's stores have read it.
-            fence_proxy_async_smem();
-            if (!named_bar_and(2, BW_CONSUMERS, !failed)) failed = true;
-            if (tid == 0 && !failed) {
-                const uint32_t stage = smem0 + (uint32_t)(s * stage_bytes);
-                const int off = c * chunk;
-                const uint32_t bytes = (uint32_t)min(chunk, a.row_bytes - off);
-                uint32_t valid;
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(valid) : "r"(stage) : "memory");
-                for (int k = 0; k < K; ++k) {
-                    if (!((valid >> k) & 1u)) continue;
-                    int sl;
-                    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * k) : "memory");
-                    bulk_s2g(a.grad_y + (size_t)sl * a.row_bytes + off, stage + BW_HDR + (uint32_t)(k * chunk), bytes);
-                }
-                bulk_commit();
-                bulk_wait_read<1>();
-                if (i > 0) mbar_arrive(empty_bar((i - 1) % BW_STAGES));
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));
         }
         if (c == a.nchunks - 1) {
             // token end: add the four warps' sums in warp order
@@ -276,9 +238,6 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
             run = 0.f;
             ++ntok;
         }
-    }
-    if constexpr (BW_BULK) {
-        if (tid == 0) bulk_wait_all();  // this CTA's grad_y stores are complete before it exits
     }
 }
 
