@@ -18,7 +18,6 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_route.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA, MOE_ERR_SCRATCH_TOO_SMALL = 0, 1, 2, 3
-MOE_DISPATCH_X_READY = 1
 MOE_STATIC_LAYOUT_SCRATCH_BYTES = 1 << 20
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_QUANT_NONE, MOE_QUANT_FP8_E4M3_B128 = 0, 1
@@ -36,7 +35,6 @@ SIGNATURES = {
     "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _Z, _P, _P]),
     "moe_dispatch": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, _P, _P]),
-    "moe_dispatch_ex": (_I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _L, ctypes.c_uint, _P, _P]),
     "moe_combine_dual_residual": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_static": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _L, _P, _P]),
     "moe_combine_fp8_dual_residual": (_I, [_P, _P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -238,10 +236,8 @@ def moe_dispatch_layout_static(topk_idx: torch.Tensor, E: int, R: int, token_pad
 
 
 def moe_dispatch(x: torch.Tensor, slot_of: torch.Tensor, cap: int, quant: int = MOE_QUANT_NONE,
-                 xd=None, xs=None, status=None, stream=None, x_ready: bool = False):
-    """Scatter rows of x [S,H] into xd [cap,H]; with FP8 also scales xs [cap,H/128].
-    x_ready=True promises that the kernel launched just before on the stream does not
-    write x (see MOE_DISPATCH_X_READY in include/moe_route.h)."""
+                 xd=None, xs=None, status=None, stream=None):
+    """Scatter rows of x [S,H] into xd [cap,H]; with FP8 also scales xs [cap,H/128]."""
     _dev(x, "x", _ACT)
     S, H = x.shape
     K = slot_of.shape[1]
@@ -259,10 +255,9 @@ def moe_dispatch(x: torch.Tensor, slot_of: torch.Tensor, cap: int, quant: int = 
         _dev(xd, "xd", (x.dtype,), (cap, H))
     if status is not None:
         _dev(status, "status", (torch.int32,))
-    flags = MOE_DISPATCH_X_READY if x_ready else 0
-    _check("moe_dispatch", lib().moe_dispatch_ex(_ptr(x), _dtype_code(x), S, H, K, _ptr(slot_of), quant,
-                                                  _ptr(xd), _ptr(xs), cap, flags, _ptr(status),
-                                                  _stream(stream, x.device)))
+    _check("moe_dispatch", lib().moe_dispatch(_ptr(x), _dtype_code(x), S, H, K, _ptr(slot_of), quant,
+                                               _ptr(xd), _ptr(xs), cap, _ptr(status),
+                                               _stream(stream, x.device)))
     return xd, xs
 
 

@@ -114,15 +114,11 @@ class MoeBuffer:
         B._check("moe_dispatch_layout", self._lib.moe_dispatch_layout(*args, self._stream(stream)))
         return self.layout
 
-    def dispatch(self, x: torch.Tensor, stream=None, x_ready: bool = False):
-        """Rows of x into the layout.  x_ready: the kernel launched just before on the
-        stream does not write x, so the dispatch may start reading x before it ends
-        (true inside step(), where the layout precedes the dispatch)."""
+    def dispatch(self, x: torch.Tensor, stream=None):
         px = self._in(x, "x", (self.dtype,), (self.S, self.H))
-        flags = B.MOE_DISPATCH_X_READY if x_ready else 0
-        B._check("moe_dispatch", self._lib.moe_dispatch_ex(px, self._dt, self.S, self.H, self.K, self._p_slot,
-                                                            self.quant, self._p_xd, self._p_xs, self.cap, flags,
-                                                            self._p_status, self._stream(stream)))
+        B._check("moe_dispatch", self._lib.moe_dispatch(px, self._dt, self.S, self.H, self.K, self._p_slot,
+                                                         self.quant, self._p_xd, self._p_xs, self.cap,
+                                                         self._p_status, self._stream(stream)))
         return self.xd, self.xs
 
     def combine(self, y: torch.Tensor, shared_out=None, residual=None, topk_w=None, stream=None):
@@ -140,7 +136,7 @@ class MoeBuffer:
         """One full pass: route, layout, dispatch, combine (y = expert outputs)."""
         self.route(logits, stream)
         self.plan(stream=stream)
-        self.dispatch(x, stream, x_ready=True)  # the layout, just before, does not write x
+        self.dispatch(x, stream)
         return self.combine(y, shared_out, residual, stream=stream)
 
     def capture(self, logits, x, y, shared_out=None, residual=None):

@@ -123,12 +123,6 @@ int moe_dispatch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int
 
 int moe_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
                  void *xd, float *xs, int64_t cap, int32_t *status, void *stream) {
-    return moe_dispatch_ex(x, dtype, S, H, K, slot_of, quant, xd, xs, cap, 0u, status, stream);
-}
-
-int moe_dispatch_ex(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
-                    void *xd, float *xs, int64_t cap, unsigned flags, int32_t *status, void *stream) {
-    if (flags & ~(unsigned)MOE_DISPATCH_X_READY) return MOE_ERR_INVALID_ARG;
     const int b = esize(dtype);
     if (S < 0 || H < 1 || K < 1 || K > MOE_MAX_TOPK || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
         return MOE_ERR_INVALID_ARG;
@@ -144,7 +138,7 @@ int moe_dispatch_ex(const void *x, int dtype, int S, int H, int K, const int32_t
     }
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
     return to_rc(moe::launch_dispatch(x, dtype, S, H, K, slot_of, quant, xd, xs, cap, status,
-                                      static_cast<cudaStream_t>(stream), (flags & MOE_DISPATCH_X_READY) != 0));
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int64_t cap,

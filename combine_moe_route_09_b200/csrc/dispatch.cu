@@ -184,7 +184,6 @@ struct Fp8Args {
     int stages;      // stages in the ring (<= DQ_MAX_STAGES)
     int obuf;        // bulk-store path: bytes per output staging buffer (codes, then scales)
     int scale_bulk;  // bulk-store path: the item's scale segment is also one bulk store per copy
-    int early;       // x is not written by the kernel launched just before: load it before waiting
 };
 
 // s = amax / 448 rounded to nearest even.  For amax >= 2^-80 this is
@@ -275,10 +274,8 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
         fence_mbar_init();
     }
     __syncthreads();
-    if (!a.early) {
-        pdl_wait();
-        pdl_trigger();
-    }
+    pdl_wait();
+    pdl_trigger();
 
     long long first, last;
     cta_range((long long)a.S * a.nchunks, first, last);
@@ -287,26 +284,6 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
     const int nb = a.H >> 7;
     if (warp == DQ_CONSUMER_WARPS) {
         // ------------------------------- producer -------------------------------
-        // Early mode: x does not depend on the kernel this one follows, so the
-        // first NS items are requested before waiting on it (the stages' full
-        // barriers get their transaction counts now and their arrivals, after
-        // the slot headers are written, below).  Slots are read after the wait.
-        int npre = 0;
-        if (a.early) {
-            npre = (int)min((long long)NS, last - first);
-            int tp = (int)(first / a.nchunks), cp = (int)(first - (long long)tp * a.nchunks);
-            for (int j = 0; j < npre; ++j, (++cp == a.nchunks ? (cp = 0, ++tp) : 0)) {
-                const int off = cp * chunk_bytes;
-                const uint32_t bytes = (uint32_t)min(chunk_bytes, row_bytes - off);
-                if (lane == 0) {
-                    mbar_expect_tx(full_bar(j), bytes);
-                    bulk_g2s(smem0 + (uint32_t)(j * a.stage) + DQ_HDR, a.x + (size_t)tp * row_bytes + off, bytes,
-                             full_bar(j));
-                }
-            }
-            pdl_wait();
-            pdl_trigger();
-        }
         // The token's slots are loaded one token ahead (lane k holds slot k).
         int t_cur = -1;
         int nxt = -1;
@@ -337,12 +314,8 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
             if (lane < K) asm volatile("st.shared.s32 [%0], %1;" ::"r"(st + 4u * lane), "r"(cur) : "memory");
             __syncwarp();
             if (lane == 0) {
-                if (i < npre) {
-                    mbar_arrive(full_bar(s));  // its data was requested before the wait
-                } else {
-                    mbar_arrive_expect_tx(full_bar(s), bytes);
-                    bulk_g2s(st + DQ_HDR, a.x + (size_t)t * row_bytes + off, bytes, full_bar(s));
-                }
+                mbar_arrive_expect_tx(full_bar(s), bytes);
+                bulk_g2s(st + DQ_HDR, a.x + (size_t)t * row_bytes + off, bytes, full_bar(s));
             }
         }
         if (lane == 0) {
@@ -358,10 +331,6 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
     // threads of a 128-channel block reduce its amax.  Codes: one 16-byte store
     // per unit and copy (a warp writes 512 contiguous bytes per copy); the
     // block's lead thread stores the scale.
-    // Early mode: the consumers let the next kernel launch only once the producer
-    // has waited (its first arrival comes after its wait), so every kernel still
-    // triggers only after the kernel before it has completed.
-    bool triggered = !a.early;
     int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
     int i = 0;
     for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
@@ -375,10 +344,6 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
             if (!named_bar_and(1, DQ_CONSUMERS, got)) break;
         } else {
             if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / NS) & 1, a.status))) break;
-        }
-        if (!triggered) {
-            pdl_trigger();
-            triggered = true;
         }
         const int col0 = c * a.bpc * 128;              // first channel of the item
         const int nch = min(a.bpc * 128, a.H - col0);  // channels in this item
@@ -519,7 +484,7 @@ static cudaError_t persistent_grid(KernelSlots<Kern> &slots, Kern kern, int thre
 
 cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of,
                             int quant, void *xd, float *xs, int64_t cap, int32_t *status,
-                            cudaStream_t st, bool x_ready) {
+                            cudaStream_t st) {
     if (S == 0) return cudaSuccess;
     const int esz = dtype == MOE_DTYPE_F32 ? 4 : 2;
     const int row_bytes = H * esz;
@@ -550,7 +515,6 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
     if (a.stages < 3) a.stages = 3;
     a.obuf = a.bpc * 128 + (a.bpc * 4 + 15) / 16 * 16;
     a.scale_bulk = (blocks % 4 == 0 && a.bpc % 4 == 0 && (reinterpret_cast<uintptr_t>(xs) & 15) == 0) ? 1 : 0;
-    a.early = x_ready ? 1 : 0;
     const bool bulk = MOE_DQ_BULK != 0;
     const size_t smem = (size_t)a.stages * a.stage + (bulk ? (size_t)DQ_OUT_BUFS * a.obuf : 0) + 2 * DQ_MAX_STAGES * 8;
     const long long nitems = (long long)S * a.nchunks;

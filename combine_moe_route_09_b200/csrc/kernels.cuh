@@ -35,7 +35,7 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
 
 cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of,
                             int quant, void *xd, float *xs, int64_t cap, int32_t *status,
-                            cudaStream_t st, bool x_ready = false);
+                            cudaStream_t st);
 
 cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_t cap,
                            const int32_t *slot_of, const float *topk_w, const void *shared_out,

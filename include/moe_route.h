@@ -230,20 +230,6 @@ MOE_API int moe_dispatch(const void *x, int dtype, int S, int H, int K, const in
                  void *xd, float *xs, int64_t cap, int32_t *status, void *stream);
 
 /*
- * moe_dispatch with flags.  MOE_DISPATCH_X_READY states that x was written
- * before the kernel launched just before this call on `stream` started (as in
- * a routing pass, where the layout kernels precede the dispatch and do not
- * touch x).  The FP8 dispatch then starts loading x while that kernel is
- * still running (programmatic dependent launch), and waits for it only
- * before reading slot_of.  Without the flag (0) it waits first.  Passing the
- * flag when the preceding kernel does write x is a race.  Unknown flag bits
- * are refused with MOE_ERR_INVALID_ARG.
- */
-#define MOE_DISPATCH_X_READY 1u
-MOE_API int moe_dispatch_ex(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
-                            void *xd, float *xs, int64_t cap, unsigned flags, int32_t *status, void *stream);
-
-/*
  * Combine: gather each token's K expert output rows, weight them by the router
  * weights, and fuse the FarSkip-Collective dual-residual epilogue.
  * [pplx] Combine: the receiver reads the payloads the routing table names and

@@ -290,28 +290,6 @@ def test_fp8_dispatch_row_shapes(H, K):
     assert np.all(host(xd.view(torch.uint8))[~used] == 0x5A) and np.all(host(xs)[~used] == -7.0)
 
 
-def test_dispatch_x_ready_right_after_layout():
-    """The dispatch that starts reading x before the layout kernel ends: new routing,
-    new activations every call, each compared with the oracle bit for bit."""
-    from combine_moe_route_09_b200.buffer import MoeBuffer
-
-    w = synth.WORKLOADS["4"].replace(S=1024)
-    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=torch.bfloat16, fp8=True, device="cuda")
-    for seed in (1, 2, 3):
-        ws = w.replace(seed=seed)
-        logits, x = synth.logits(ws), synth.activations(ws)
-        buf.route(dev(logits))
-        buf.plan()
-        xd, xs = buf.dispatch(dev(x), x_ready=True)
-        idx, _ = oracle.route_topk(logits, w.K)
-        lay = oracle.layout(idx, w.E, w.R, w.P)
-        ref_xd, ref_xs = oracle.dispatch(x, lay["slot_of"], lay["cap"], quant=oracle.QUANT_FP8_E4M3_B128)
-        np.testing.assert_array_equal(host(buf.layout.slot_of), lay["slot_of"])
-        np.testing.assert_array_equal(host(xd), ref_xd)
-        np.testing.assert_array_equal(host(xs), ref_xs)
-    assert buf.read_status() == 0
-
-
 def test_fp8_dispatch_scale_rows_not_16_byte_aligned():
     """A scale array whose base is only 4-byte aligned: scales are stored per block."""
     rng = np.random.default_rng(5)
