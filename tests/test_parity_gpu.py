@@ -157,3 +157,41 @@ def test_captured_step_replays_the_pass(case):
         np.testing.assert_array_equal(host(buf.xd)[valid], ref["xd"][valid])
         assert_act_close(host(buf.out), ref["out"], "residual_out", extra_abs=weight_slack)
         assert buf.read_status() == 0
+
+
+@pytest.mark.parametrize("name", ["3", "4"])
+def test_captured_step_with_new_inputs(name):
+    """A captured step replayed after its inputs were refilled in place with another
+    draw (different routing, different activations) gives that draw's pass."""
+    w = synth.WORKLOADS[name]
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8")
+    first = workload_inputs(w)
+    args = {k: dev(v) for k, v in first.items()}
+    order = ["logits", "x", "y"] + (["shared", "residual"] if w.fused else [])
+    buf.step(*[args[k] for k in order])
+    torch.cuda.synchronize()
+    graph = buf.capture(*[args[k] for k in order])
+    w2 = w.replace(seed=w.seed + 1000)
+    second = workload_inputs(w2)
+    for k in order:
+        args[k].copy_(dev(second[k]))
+    graph.replay()
+    torch.cuda.synchronize()
+    idx, wt = oracle.route_topk(second["logits"], w.K)
+    lay = oracle.layout(idx, w.E, w.R, w.P)
+    q = oracle.QUANT_FP8_E4M3_B128 if w.quant == "fp8" else oracle.QUANT_NONE
+    xd, xs = oracle.dispatch(second["x"], lay["slot_of"], lay["cap"], quant=q)
+    out, rnr = oracle.combine(second["y"], lay["slot_of"], wt, second.get("shared"), second.get("residual"))
+    assert not np.array_equal(idx, oracle.route_topk(first["logits"], w.K)[0])  # the routing did change
+    np.testing.assert_array_equal(host(buf.topk_idx), idx)
+    _check_layout(buf.layout, lay)
+    valid = lay["row_src"] >= 0
+    np.testing.assert_array_equal(host(buf.xd)[valid], xd[valid])
+    if q == oracle.QUANT_FP8_E4M3_B128:
+        np.testing.assert_array_equal(host(buf.xs)[valid], xs[valid])
+    slack = 2e-5 * abs_weighted_sum(second["y"], lay["slot_of"], wt)
+    assert_act_close(host(buf.out), out, "residual_out", extra_abs=slack)
+    if w.fused:
+        assert_act_close(host(buf.out_no_routed), rnr, "residual_no_routed_out")
+    assert buf.read_status() == 0
