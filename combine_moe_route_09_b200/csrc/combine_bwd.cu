@@ -24,21 +24,7 @@
 
 namespace moe {
 
-#ifndef MOE_BW_STAGES
-#define MOE_BW_STAGES 4
-#endif
-#ifndef MOE_BW_STAGE_OUT
-#define MOE_BW_STAGE_OUT 0
-#endif
-#ifndef MOE_BW_OUT_BUFS
-#define MOE_BW_OUT_BUFS 2
-#endif
-constexpr int BW_STAGES = MOE_BW_STAGES;
-// STAGE_OUT: grad_y goes through OUT_BUFS shared-memory staging buffers of K
-// chunks and leaves as K bulk stores issued by one thread (instead of
-// per-thread 16-byte stores).
-constexpr bool BW_STAGE_OUT = MOE_BW_STAGE_OUT != 0;
-constexpr int BW_OUT_BUFS = MOE_BW_OUT_BUFS;
+constexpr int BW_STAGES = 4;
 constexpr int BW_CONSUMER_WARPS = 4;
 constexpr int BW_CONSUMERS = BW_CONSUMER_WARPS * 32;
 constexpr int BW_THREADS = BW_CONSUMERS + 32;
@@ -92,13 +78,11 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     using V = BVec<F32>;
     constexpr int N = V::N;
     extern __shared__ __align__(128) uint8_t smem[];
-    // [STAGES][header (mask, weights, slots) | K y chunks | g chunk | gn chunk]
-    // | STAGE_OUT: [OUT_BUFS][K grad_y chunks] | barriers | per-warp dot sums [2][4][32]
+    // [STAGES][header (mask, weights, slots) | K y chunks | g chunk | gn chunk] | barriers |
+    // per-warp dot sums [2][4][32]
     const int K = a.K, chunk = a.chunk;
     const int stage_bytes = BW_HDR + (K + 2) * chunk;
-    const int out_bytes = BW_STAGE_OUT ? K * chunk : 0;
-    const uint32_t obuf0 = smem_addr(smem) + (uint32_t)(BW_STAGES * stage_bytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + BW_STAGES * stage_bytes + BW_OUT_BUFS * out_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + BW_STAGES * stage_bytes);
     float *wsum = reinterpret_cast<float *>(bars + 2 * BW_STAGES);
     const uint32_t smem0 = smem_addr(smem);
     const uint32_t bar0 = smem_addr(bars);
@@ -187,16 +171,7 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     int i = 0, t = t_first, c = 0, ntok = 0;
     for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
         const int s = i % BW_STAGES;
-        if constexpr (BW_STAGE_OUT) {
-            // all consumers agree on a timeout; the issuing thread first lets the
-            // stores that last read this item's staging buffer finish reading it
-            const bool got = !failed && mbar_wait(full_bar(s), (i / BW_STAGES) & 1, a.status);
-            if (tid == 0) bulk_wait_read<BW_OUT_BUFS - 1>();
-            if (!named_bar_and(3, BW_CONSUMERS, got)) failed = true;
-        } else {
-            if (!failed) failed = !__all_sync(FULL, mbar_wait(full_bar(s), (i / BW_STAGES) & 1, a.status));
-        }
-        const uint32_t ob = obuf0 + (uint32_t)((i % BW_OUT_BUFS) * out_bytes);
+        if (!failed) failed = !__all_sync(FULL, mbar_wait(full_bar(s), (i / BW_STAGES) & 1, a.status));
         if (!failed) {
             const int off = c * chunk;
             const int bytes = min(chunk, a.row_bytes - off);
@@ -235,13 +210,9 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
                             p = __fmaf_rn(yf[e], gf[e], p);
                             gy[e] = __fmul_rn(wk, gf[e]);
                         }
-                        if constexpr (BW_STAGE_OUT) {
-                            sts128(ob + (uint32_t)(k * chunk + ub), V::pack(gy));
-                        } else {
-                            int sl;
-                            asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * k) : "memory");
-                            st_v4(a.grad_y + (size_t)sl * a.row_bytes + off + ub, V::pack(gy));
-                        }
+                        int sl;
+                        asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * k) : "memory");
+                        st_v4(a.grad_y + (size_t)sl * a.row_bytes + off + ub, V::pack(gy));
                     }
                     // fixed xor tree: every lane ends with the warp's partial for pair k
 #pragma unroll
@@ -249,30 +220,8 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
                     if (lane == k) run += p;
                 }
             }
-            if constexpr (BW_STAGE_OUT) {
-                // the slots and mask are needed after the stage is freed: warp 0 keeps them
-                uint32_t valid2;
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(valid2) : "r"(stage) : "memory");
-                int sl = -1;
-                if (warp == 0 && lane < K)
-                    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(sl) : "r"(stage + 132u + 4u * lane) : "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-                fence_proxy_async_smem();
-                named_bar(2, BW_CONSUMERS);
-                if (warp == 0) {
-                    for (int k = 0; k < K; ++k) {
-                        const int slk = __shfl_sync(FULL, sl, k);
-                        if (lane == 0 && ((valid2 >> k) & 1u))
-                            bulk_s2g(a.grad_y + (size_t)slk * a.row_bytes + off, ob + (uint32_t)(k * chunk),
-                                     (uint32_t)bytes);
-                    }
-                    if (lane == 0) bulk_commit();
-                }
-            } else {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));
         }
         if (c == a.nchunks - 1) {
             // token end: add the four warps' sums in warp order
@@ -290,16 +239,12 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
             ++ntok;
         }
     }
-    if constexpr (BW_STAGE_OUT) {
-        if (tid == 0) bulk_wait_all();  // this CTA's grad_y stores are complete before it exits
-    }
 }
 
 template <bool F32, bool GN, bool SKIP>
 static cudaError_t launch_bwd(const CombineBwdArgs &a, cudaStream_t st) {
     auto kern = combine_bwd_kernel<F32, GN, SKIP>;
-    const size_t smem = (size_t)BW_STAGES * (BW_HDR + (a.K + 2) * a.chunk) +
-                        (BW_STAGE_OUT ? (size_t)BW_OUT_BUFS * a.K * a.chunk : 0) + 2 * BW_STAGES * 8 +
+    const size_t smem = (size_t)BW_STAGES * (BW_HDR + (a.K + 2) * a.chunk) + 2 * BW_STAGES * 8 +
                         2 * BW_CONSUMER_WARPS * 32 * sizeof(float);
     static KernelSlots<decltype(kern)> slots;
     int sms = 0, per_sm = 0;
@@ -340,9 +285,7 @@ cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y
     a.K = K;
     a.row_bytes = H * (f32 ? 4 : 2);
     int chunk = BW_MAX_CHUNK;
-    while (chunk > 256 && BW_STAGES * (BW_HDR + (K + 2) * chunk) + (BW_STAGE_OUT ? BW_OUT_BUFS * K * chunk : 0) >
-                              BW_SMEM_BUDGET)
-        chunk >>= 1;
+    while (chunk > 256 && BW_STAGES * (BW_HDR + (K + 2) * chunk) > BW_SMEM_BUDGET) chunk >>= 1;
     a.chunk = chunk < a.row_bytes ? chunk : a.row_bytes;
     a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
     return f32 ? launch_bwd_dt<true>(a, st) : launch_bwd_dt<false>(a, st);
