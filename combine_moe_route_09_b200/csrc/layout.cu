@@ -522,7 +522,10 @@ __global__ void __launch_bounds__(LT_THREADS)
 #endif
 constexpr int LC_WARPS = MOE_LC_WARPS;
 constexpr int LC_THREADS = LC_WARPS * 32;
-constexpr int LC_ITEMS = 4;
+#ifndef MOE_LC_ITEMS
+#define MOE_LC_ITEMS 4
+#endif
+constexpr int LC_ITEMS = MOE_LC_ITEMS;
 constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // 2048 pairs per CTA
 // 16 CTAs: above the portable cluster size of 8, allowed per function (the
 // layout falls back to the other paths where the device refuses it).  In the
