@@ -328,9 +328,10 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
     // ------------------------------- consumers -------------------------------
     // Thread tid owns two 16-channel units of the item, channels
     // [16 tid + 2048 u, +16) for u = 0, 1 (two independent chains); the 8
-    // threads of a 128-channel block reduce its amax.  Codes: one 16-byte store
-    // per unit and copy (a warp writes 512 contiguous bytes per copy); the
-    // block's lead thread stores the scale.
+    // threads of a 128-channel block reduce its amax.  BULK: the codes and the
+    // blocks' scales go to a staging buffer and leave as bulk stores; otherwise
+    // one 16-byte store per unit and copy (a warp writes 512 contiguous bytes
+    // per copy) and the block's lead thread stores the scale.
     int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
     int i = 0;
     for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {

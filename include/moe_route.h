@@ -12,6 +12,13 @@
  *   moe_combine_dual_residual gather + top-K weighted sum back to token order,
  *                             fused with the FarSkip-Collective dual residual
  *
+ * and around them: the backward of each step (moe_combine_dual_residual_backward,
+ * moe_dispatch_backward, moe_route_topk_backward), the combine over FP8 expert
+ * outputs (moe_combine_fp8_dual_residual), the routing weights in dispatched
+ * order (moe_dispatch_route_weights), a sigmoid / selection-bias /
+ * group-limited router (moe_route_sigmoid_grouped), an allocation-free layout
+ * (moe_dispatch_layout_static) and host-side queries.
+ *
  * Sources (page title, section):
  *   [pplx]    "Efficient and portable mixture-of-experts communication"
  *             (Perplexity, pplx-kernels): Introduction; Portable Kernels;
@@ -30,8 +37,10 @@
  *
  * Conventions for every entry point
  *   - Every pointer except `stream` and those marked "host" is DEVICE memory
- *     that the caller allocated and owns.  The library allocates nothing,
- *     keeps no state between calls, and never synchronises with the host:
+ *     that the caller allocated and owns.  The library allocates nothing and
+ *     keeps no data between calls (only per-process launch settings: kernel
+ *     attributes and occupancy answers, plus the fixed scratch array of
+ *     moe_dispatch_layout_static), and it never synchronises with the host:
  *     all work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns once it is enqueued.
  *   - Arrays are dense row-major.  Activation buffers (x, xd, y, shared_out,
