@@ -153,7 +153,10 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
 #endif
 constexpr int DQ_MAX_STAGES = 8;
 constexpr int DQ_STAGE_BUDGET = MOE_DQ_STAGE_BUDGET;         // bytes of input ring per CTA
-constexpr int DQ_CONSUMER_WARPS = 4;
+#ifndef MOE_DQ_CONSUMER_WARPS
+#define MOE_DQ_CONSUMER_WARPS 4
+#endif
+constexpr int DQ_CONSUMER_WARPS = MOE_DQ_CONSUMER_WARPS;
 constexpr int DQ_CONSUMERS = DQ_CONSUMER_WARPS * 32;
 constexpr int DQ_THREADS = DQ_CONSUMERS + 32;
 constexpr int DQ_UNIT = 16;                                  // channels of one thread unit
