@@ -63,11 +63,12 @@ __device__ __forceinline__ void decode8(uint32_t lo, uint32_t hi, float (&f)[8])
     }
 }
 
-template <bool F32, bool HAS_SH, bool HAS_RS, bool HAS_RNR>
+// KT: K known at compile time (0 = runtime K); with it the per-pair loop unrolls.
+template <bool F32, bool HAS_SH, bool HAS_RS, bool HAS_RNR, int KT>
 __global__ void __launch_bounds__(C8_THREADS) combine_fp8_kernel(const CombineFp8Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     // [STAGES][header | K code chunks (cch B) | K scale segments (cch/32 B) | shared | residual]
-    const int K = a.K, cch = a.cch;
+    const int K = KT > 0 ? KT : a.K, cch = a.cch;
     const int seg = cch / 32;  // scale bytes per item and row
     const int obytes = cch * a.ob;
     const int stage_bytes = C8_HDR + K * cch + K * seg + 2 * obytes;
@@ -172,6 +173,8 @@ __global__ void __launch_bounds__(C8_THREADS) combine_fp8_kernel(const CombineFp
             float acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+            constexpr int KU = KT > 0 ? KT : 1;
+#pragma unroll(KU)
             for (int k = 0; k < K; ++k) {
                 if (!((valid >> k) & 1u)) continue;
                 float wk, sc;
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(C8_THREADS) combine_fp8_kernel(const CombineFp
 
 template <bool F32, bool SH, bool RS, bool RNR>
 static cudaError_t launch_c8(const CombineFp8Args &a, cudaStream_t st) {
-    auto kern = combine_fp8_kernel<F32, SH, RS, RNR>;
+    auto kern = a.K == 8 ? combine_fp8_kernel<F32, SH, RS, RNR, 8> : combine_fp8_kernel<F32, SH, RS, RNR, 0>;
     const int seg = a.cch / 32;
     const size_t smem = (size_t)C8_STAGES * (C8_HDR + a.K * (a.cch + seg) + 2 * a.cch * a.ob) + 2 * C8_STAGES * 8;
     static KernelSlots<decltype(kern)> slots;
