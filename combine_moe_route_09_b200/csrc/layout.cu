@@ -14,7 +14,7 @@
 // spin-waits and no global atomics except one arrival counter:
 //
 //  layout_hist   one CTA per tile of LT_TILE pairs.  Each warp ranks its 32
-//                pairs by expert with __match_any_sync (peers share an expert;
+//                pairs by expert (peers sharing an expert are found with one ballot per id bit;
 //                the lowest peer adds the group size to the warp's private
 //                shared-memory histogram), so the tile histogram is built
 //                without atomics.  The CTA writes it to hist[tile][E], then
@@ -42,6 +42,24 @@ struct LayoutHeader {
 };
 
 __device__ __forceinline__ int pad_count(int c, int P) { return P > 0 ? ((c + P - 1) / P) * P : c; }
+
+// Lanes of the warp holding the same expert id as this lane (e = -1: none).
+// One ballot per bit of the id (ids below 2^nbits) plus one for validity: a
+// fixed, short sequence, where __match_any_sync takes longer the more
+// distinct values the warp holds.
+__device__ __forceinline__ unsigned expert_peers(int e, int nbits) {
+    unsigned peers = __ballot_sync(FULL, e >= 0);
+    if (e < 0) peers = ~peers;
+    for (int b = 0; b < nbits; ++b) {
+        const bool bit = (e >> b) & 1;
+        const unsigned m = __ballot_sync(FULL, bit);
+        peers &= bit ? m : ~m;
+    }
+    return peers;
+}
+
+// Bits that cover every expert id below E.
+__device__ __forceinline__ int expert_bits(int E) { return E > 1 ? 32 - __clz(E - 1) : 0; }
 
 __global__ void __launch_bounds__(LT_THREADS)
     layout_hist_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P,
@@ -77,7 +95,7 @@ __global__ void __launch_bounds__(LT_THREADS)
             bad = true;
             e = -1;
         }
-        const unsigned peers = __match_any_sync(FULL, e);
+        const unsigned peers = expert_peers(e, expert_bits(E));
         if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] += (uint16_t)__popc(peers);
         __syncwarp();
     }
@@ -205,7 +223,7 @@ __global__ void __launch_bounds__(LT_THREADS)
     for (int it = 0; it < LT_ITEMS; ++it) {
         int e = ev[it];
         if (e < 0 || e >= E) e = -1;
-        const unsigned peers = __match_any_sync(FULL, e);
+        const unsigned peers = expert_peers(e, expert_bits(E));
         const int before = e >= 0 ? (int)whist[w * E + e] : 0;
         __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
@@ -327,7 +345,7 @@ __device__ __forceinline__ bool rank_tile(const int32_t *topk_idx, int npairs, i
             bad = true;
             e = -1;
         }
-        const unsigned peers = __match_any_sync(FULL, e);
+        const unsigned peers = expert_peers(e, expert_bits(E));
         const int before = e >= 0 ? (int)whist[w * E + e] : 0;
         __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1) whist[w * E + e] = (uint16_t)(before + __popc(peers));
@@ -506,12 +524,10 @@ __global__ void __launch_bounds__(LT_THREADS)
 // ------------------------------------------------------------------------------------------
 // Cluster layout: up to LC_MAX_CTAS tiles of LC_TILE pairs, one CTA each, all
 // in one thread-block cluster (E <= LC_THREADS).  Each CTA ranks its tile (as
-// above), keeps the tile histogram in its own shared memory, and after one
-// hardware cluster barrier reads the other CTAs' histograms through
-// distributed shared memory: the per-expert totals and the counts of the tiles
-// below it.  No global scratch, no atomics, no spin-wait.  A second cluster
-// barrier (arrive after the remote reads, wait before exit) keeps every CTA's
-// shared memory alive until the others have read it.
+// above) and stores its tile histogram into every CTA's shared memory
+// (distributed shared memory); after one hardware cluster barrier each CTA
+// has all tiles' counts locally: the per-expert totals and the counts of the
+// tiles below it.  No global scratch, no atomics, no spin-wait.
 // ------------------------------------------------------------------------------------------
 
 #ifndef MOE_LC_WARPS
@@ -538,7 +554,8 @@ __global__ void __launch_bounds__(LC_THREADS)
                           int32_t *__restrict__ rank_offsets, int32_t *__restrict__ slot_of,
                           int32_t *__restrict__ row_src, int32_t *status) {
     extern __shared__ __align__(16) uint8_t lc_smem[];
-    int *thist = reinterpret_cast<int *>(lc_smem);             // [E] this tile's counts (read cluster-wide)
+    int *allh = reinterpret_cast<int *>(lc_smem);              // [LC_MAX_CTAS][E] every tile's counts, pushed by its CTA
+    int *thist = allh + LC_MAX_CTAS * E;                        // [E] this tile's counts
     int *s_tot = thist + E;                                     // [E] totals
     int *s_base = s_tot + E;                                    // [E] first row of this tile's pairs, per expert
     int *s_off = s_base + E;                                    // [E + 1] padded offsets
@@ -574,7 +591,7 @@ __global__ void __launch_bounds__(LC_THREADS)
             bad = true;
             e = -1;
         }
-        const unsigned peers = __match_any_sync(FULL, e);
+        const unsigned peers = expert_peers(e, expert_bits(E));
         const int before = e >= 0 ? (int)whist[w * WS + e] : 0;
         __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1) whist[w * WS + e] = (uint16_t)(before + __popc(peers));
@@ -614,26 +631,30 @@ __global__ void __launch_bounds__(LC_THREADS)
             }
         }
     }
+    __syncthreads();
+    // push this tile's counts into row `me` of every CTA's allh (stores into the
+    // cluster's distributed shared memory), then one cluster barrier: after it
+    // every CTA holds all tiles' counts locally, and no CTA touches another's
+    // shared memory again, so none has to wait for the others before exiting
+    const uint32_t ah = smem_addr(allh) + 4u * me * (uint32_t)E;
+    for (int idx = tid; idx < C * E; idx += LC_THREADS) {
+        const int c = idx / E, e = idx - c * E;
+        st_cluster_s32(cluster_map(ah + 4u * e, (uint32_t)c), thist[e]);
+    }
     cluster_arrive();
-    cluster_wait();  // every tile histogram of the cluster is complete and visible
+    cluster_wait();
 
-    // ---- totals and the count of the tiles below this one, from all CTAs' thist ----
-    const uint32_t th = smem_addr(thist);
+    // ---- totals and the count of the tiles below this one ----
     for (int e = tid; e < E; e += LC_THREADS) {
-        int v[LC_MAX_CTAS];
-#pragma unroll
-        for (int c = 0; c < LC_MAX_CTAS; ++c)  // independent remote loads, all in flight
-            v[c] = c < C ? ld_cluster_s32(cluster_map(th + 4u * e, (uint32_t)c)) : 0;
         int all = 0, below = 0;
-#pragma unroll
-        for (int c = 0; c < LC_MAX_CTAS; ++c) {
-            all += v[c];
-            below += (uint32_t)c < me ? v[c] : 0;
+        for (int c = 0; c < C; ++c) {
+            const int v = allh[c * E + e];
+            all += v;
+            below += (uint32_t)c < me ? v : 0;
         }
         s_tot[e] = all;
         s_base[e] = below;
     }
-    cluster_arrive_relaxed();  // done reading the others' shared memory (waited for before exit)
     __syncthreads();
 
     // ---- exclusive scan of the padded counts over experts (one expert per thread) ----
@@ -701,7 +722,6 @@ __global__ void __launch_bounds__(LC_THREADS)
     }
     for (int64_t r = (int64_t)s_off[E] + (int64_t)tile * LC_THREADS + tid; r < cap; r += (int64_t)C * LC_THREADS)
         row_src[r] = -1;
-    cluster_wait();  // the other CTAs have finished reading this CTA's thist
 }
 
 static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, int E, int R, int P, int64_t cap,
@@ -711,7 +731,8 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     *launched = false;
     const int C = (npairs + LC_TILE - 1) / LC_TILE;
     if (C < 1 || C > LC_MAX_CTAS || E > LC_THREADS) return cudaSuccess;  // not launched
-    const size_t smem = (size_t)(4 * E + 4) * sizeof(int) + (size_t)LC_WARPS * (E + 2) * sizeof(uint16_t);
+    // ints: allh [LC_MAX_CTAS][E], thist, s_tot, s_base [E] each, s_off [E + 1], 3 of padding; then whist
+    const size_t smem = (size_t)((LC_MAX_CTAS + 4) * E + 4) * sizeof(int) + (size_t)LC_WARPS * (E + 2) * sizeof(uint16_t);
     static KernelSlots<decltype(&layout_cluster_kernel)> slots;
     int sms = 0, per_sm = 0;
     cudaError_t e = slots.prepare(&layout_cluster_kernel, LC_THREADS, smem, &sms, &per_sm);
