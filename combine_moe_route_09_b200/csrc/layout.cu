@@ -559,10 +559,14 @@ __global__ void __launch_bounds__(LC_THREADS)
     int *s_tot = thist + E;                                     // [E] totals
     int *s_base = s_tot + E;                                    // [E] first row of this tile's pairs, per expert
     int *s_off = s_base + E;                                    // [E + 1] padded offsets
+    int *s_lbase = s_off + E + 1;                               // [E] first position of expert e in the tile's sorted order
+    int *loc_p = s_lbase + E;                                   // [LC_TILE] the tile's pairs sorted by (expert, pair)
+    int *loc_s = loc_p + LC_TILE;                               // [LC_TILE] their slots
     // [LC_WARPS][E + 2]: the padded row stride moves each warp's row by one bank
-    uint16_t *whist = reinterpret_cast<uint16_t *>(s_off + E + 1 + 3);
+    uint16_t *whist = reinterpret_cast<uint16_t *>(loc_s + LC_TILE + 3);
     const int WS = E + 2;
     __shared__ int s_wsum[LC_WARPS];
+    __shared__ int s_lsum[LC_WARPS];
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int C = gridDim.x;
@@ -657,32 +661,51 @@ __global__ void __launch_bounds__(LC_THREADS)
     }
     __syncthreads();
 
-    // ---- exclusive scan of the padded counts over experts (one expert per thread) ----
+    // ---- exclusive scans over experts (one expert per thread): the padded
+    // totals give the offsets, this tile's counts give its local sorted order ----
     const int pc = tid < E ? pad_count(s_tot[tid], P) : 0;
-    int incl = pc;
+    const int lc = tid < E ? thist[tid] : 0;
+    int incl = pc, lincl = lc;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(FULL, incl, off);
-        if (lane >= off) incl += o;
+        const int lo = __shfl_up_sync(FULL, lincl, off);
+        if (lane >= off) {
+            incl += o;
+            lincl += lo;
+        }
     }
-    if (lane == 31) s_wsum[w] = incl;
+    if (lane == 31) {
+        s_wsum[w] = incl;
+        s_lsum[w] = lincl;
+    }
     __syncthreads();
     if (w == 0) {
         int v = lane < LC_WARPS ? s_wsum[lane] : 0;
+        int lv = lane < LC_WARPS ? s_lsum[lane] : 0;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(FULL, v, off);
-            if (lane >= off) v += o;
+            const int lo = __shfl_up_sync(FULL, lv, off);
+            if (lane >= off) {
+                v += o;
+                lv += lo;
+            }
         }
-        if (lane < LC_WARPS) s_wsum[lane] = v;  // inclusive over warps
+        if (lane < LC_WARPS) {
+            s_wsum[lane] = v;  // inclusive over warps
+            s_lsum[lane] = lv;
+        }
     }
     __syncthreads();
     if (tid < E) {
         const int off = incl - pc + (w > 0 ? s_wsum[w - 1] : 0);
         s_off[tid] = off;
         s_base[tid] += off;
+        s_lbase[tid] = lincl - lc + (w > 0 ? s_lsum[w - 1] : 0);
     }
     if (tid == 0) s_off[E] = s_wsum[LC_WARPS - 1];
+    const int nsorted = s_lsum[LC_WARPS - 1];  // this tile's pairs with a valid expert
     __syncthreads();
     if (me == 0) {
         for (int e = tid; e <= E; e += LC_THREADS) offsets[e] = s_off[e];
@@ -701,16 +724,26 @@ __global__ void __launch_bounds__(LC_THREADS)
         const int e = my_e[it];
         int sl = -1;
         if (e >= 0) {
-            sl = s_base[e] + whist[w * WS + e] + my_r[it];
+            const int within = whist[w * WS + e] + my_r[it];  // earlier pairs of e in this tile
+            sl = s_base[e] + within;
             if ((int64_t)sl >= cap) {
                 sl = -1;
                 over = true;
             }
+            const int lp = s_lbase[e] + within;
+            loc_p[lp] = p;
+            loc_s[lp] = sl;
         }
         slot_of[p] = sl;
-        if (sl >= 0) row_src[sl] = p;
     }
     if (over) set_status(status, MOE_STATUS_OVERFLOW);
+    __syncthreads();
+    // row_src in slot order: consecutive threads write the consecutive rows of
+    // each expert's run, so a warp's stores share sectors
+    for (int j = tid; j < nsorted; j += LC_THREADS) {
+        const int sl = loc_s[j];
+        if (sl >= 0) row_src[sl] = loc_p[j];
+    }
 
     // ---- padding rows (one warp per expert) and rows past the layout ----
     const int gw = tile * LC_WARPS + w, nw = C * LC_WARPS;
@@ -731,8 +764,10 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     *launched = false;
     const int C = (npairs + LC_TILE - 1) / LC_TILE;
     if (C < 1 || C > LC_MAX_CTAS || E > LC_THREADS) return cudaSuccess;  // not launched
-    // ints: allh [LC_MAX_CTAS][E], thist, s_tot, s_base [E] each, s_off [E + 1], 3 of padding; then whist
-    const size_t smem = (size_t)((LC_MAX_CTAS + 4) * E + 4) * sizeof(int) + (size_t)LC_WARPS * (E + 2) * sizeof(uint16_t);
+    // ints: allh [LC_MAX_CTAS][E], thist, s_tot, s_base [E] each, s_off [E + 1], s_lbase [E],
+    // loc_p, loc_s [LC_TILE] each, 3 of padding; then whist
+    const size_t smem = (size_t)((LC_MAX_CTAS + 5) * E + 2 * LC_TILE + 4) * sizeof(int) +
+                        (size_t)LC_WARPS * (E + 2) * sizeof(uint16_t);
     static KernelSlots<decltype(&layout_cluster_kernel)> slots;
     int sms = 0, per_sm = 0;
     cudaError_t e = slots.prepare(&layout_cluster_kernel, LC_THREADS, smem, &sms, &per_sm);
