@@ -171,9 +171,6 @@ constexpr int DQ_HDR = 128;                                  // per-stage header
 #define MOE_DQ_OUT_BUFS 2
 #endif
 constexpr int DQ_OUT_BUFS = MOE_DQ_OUT_BUFS;                 // bulk-store path: output staging buffers
-#ifndef MOE_DQ_EVICT_FIRST
-#define MOE_DQ_EVICT_FIRST 0
-#endif
 
 struct Fp8Args {
     const uint8_t *x;
@@ -430,22 +427,12 @@ __global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kern
             named_bar(2, DQ_CONSUMERS);
             const int nblk = nch >> 7;
             if (warp == 0) {
-#if MOE_DQ_EVICT_FIRST
-                const uint64_t pol = l2_policy_evict_first();
-#endif
                 for (int k = 0; k < K; ++k) {
                     const int sl = __shfl_sync(FULL, myslot, k);
                     if (lane == 0 && sl >= 0) {
-#if MOE_DQ_EVICT_FIRST
-                        bulk_s2g_hint(a.xd + (size_t)sl * a.H + col0, ob, (uint32_t)nch, pol);
-                        if (a.scale_bulk)
-                            bulk_s2g_hint(a.xs + (size_t)sl * nb + (col0 >> 7), ob + (uint32_t)cbytes,
-                                          (uint32_t)nblk * 4u, pol);
-#else
                         bulk_s2g(a.xd + (size_t)sl * a.H + col0, ob, (uint32_t)nch);
                         if (a.scale_bulk)
                             bulk_s2g(a.xs + (size_t)sl * nb + (col0 >> 7), ob + (uint32_t)cbytes, (uint32_t)nblk * 4u);
-#endif
                     }
                 }
                 if (lane == 0) bulk_commit();
