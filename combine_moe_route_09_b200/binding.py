@@ -30,6 +30,7 @@ _P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 SIGNATURES = {
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_dispatch_layout_kernels": (_I, [_I, _I, _I]),
+    "moe_selftest_wait_timeout": (_I, [_I, ctypes.c_ulonglong, _P, _P, _P]),
     "moe_dispatch_route_weights": (_I, [_P, _P, _I, _I, _L, _P, _P, _P]),
     "moe_route_sigmoid_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "moe_dispatch_layout_workspace": (_Z, [_I, _I, _I]),
@@ -121,6 +122,16 @@ def moe_route_topk(logits: torch.Tensor, K: int, topk_idx=None, topk_w=None, str
     _check("moe_route_topk", lib().moe_route_topk(_ptr(logits), S, E, K, _ptr(topk_idx), _ptr(topk_w),
                                                    _stream(stream, logits.device)))
     return topk_idx, topk_w
+
+
+def moe_selftest_wait_timeout(which: int, limit_ns: int, status: torch.Tensor, flag=None, stream=None):
+    """Runs one bounded wait that nothing completes (0: mbarrier, 1: flag poll); it sets the
+    timeout bit in `status` (device int32 [1]) and returns."""
+    _dev(status, "status", (torch.int32,), (1,))
+    if flag is not None:
+        _dev(flag, "flag", (torch.int32,), (1,))
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(
+        which, limit_ns, _ptr(status), _ptr(flag), _stream(stream, status.device)))
 
 
 def moe_dispatch_layout_kernels(S: int, E: int, K: int) -> int:

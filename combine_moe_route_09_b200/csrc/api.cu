@@ -57,6 +57,13 @@ int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, 
                                         static_cast<cudaStream_t>(stream), current_sms()));
 }
 
+int moe_selftest_wait_timeout(int which, unsigned long long limit_ns, int32_t *status, uint32_t *flag,
+                              void *stream) {
+    if ((which != 0 && which != 1) || limit_ns < 1 || limit_ns > 1000000000ull) return MOE_ERR_INVALID_ARG;
+    if (!status || !aligned(status, 4) || (which == 1 && (!flag || !aligned(flag, 4)))) return MOE_ERR_INVALID_ARG;
+    return to_rc(moe::launch_wait_selftest(which, limit_ns, status, flag, static_cast<cudaStream_t>(stream)));
+}
+
 int moe_dispatch_layout_kernels(int S, int E, int K) {
     if (S < 1 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK || (int64_t)S * K >= ((int64_t)1 << 31)) return 0;
     return moe::layout_kernel_count(S, E, K);

@@ -56,6 +56,9 @@ cudaError_t launch_route_sigmoid_grouped(const float *logits, const float *bias,
                                          int topk_group, int normalize, float scale, int32_t *idx, float *w,
                                          cudaStream_t st, int sms);
 
+cudaError_t launch_wait_selftest(int which, unsigned long long limit_ns, int32_t *status, const unsigned *flag,
+                                 cudaStream_t st);
+
 // Kernels moe_dispatch_layout launches for these sizes on the current device (1 or 2; -1: CUDA error).
 int layout_kernel_count(int S, int E, int K);
 

@@ -307,15 +307,7 @@ __device__ bool grid_barrier(LayoutHeader *hdr, int32_t *status) {
             __threadfence();
             atomicExch(&hdr->gen, gen + 1u);
         } else {
-            const unsigned long long t0 = globaltimer();
-            while (*(volatile unsigned *)&hdr->gen == gen) {
-                if (globaltimer() - t0 > MOE_WAIT_NS) {
-                    set_status(status, MOE_STATUS_TIMEOUT);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(64);
-            }
+            ok = wait_changed_for(&hdr->gen, gen, status, MOE_WAIT_NS) ? 1 : 0;
         }
         __threadfence();
         s_ok = ok;

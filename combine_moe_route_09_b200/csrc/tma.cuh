@@ -55,16 +55,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Waits for the phase with the given parity to complete; false on timeout
-// (MOE_STATUS_TIMEOUT is then set).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+// Waits for the phase with the given parity to complete, for at most
+// limit_ns; false on timeout (MOE_STATUS_TIMEOUT is then set).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int32_t *status,
+                                              unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > MOE_WAIT_NS) {
+        if (globaltimer() - t0 > limit_ns) {
             set_status(status, MOE_STATUS_TIMEOUT);
             return false;
         }
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+    return mbar_wait_for(bar, parity, status, MOE_WAIT_NS);
+}
+
+// Polls a global word until it differs from `old`, for at most limit_ns (with
+// a short sleep between reads); false on timeout (MOE_STATUS_TIMEOUT is set).
+__device__ __forceinline__ bool wait_changed_for(const unsigned *p, unsigned old, int32_t *status,
+                                                 unsigned long long limit_ns) {
+    const unsigned long long t0 = globaltimer();
+    while (*(const volatile unsigned *)p == old) {
+        if (globaltimer() - t0 > limit_ns) {
+            set_status(status, MOE_STATUS_TIMEOUT);
+            return false;
+        }
+        __nanosleep(64);
     }
     return true;
 }

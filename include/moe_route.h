@@ -118,6 +118,18 @@ MOE_API int moe_route_topk(const float *logits, int S, int E, int K, int32_t *to
                    void *stream);
 
 /*
+ * Self-test of the library's failure detection (no counterpart on the pages).
+ * Runs one bounded wait that nothing will complete -- which = 0: an mbarrier
+ * phase with no arrival; which = 1: a poll of *flag (device, 4 bytes, not
+ * written by anyone while the test runs) -- with a limit of limit_ns
+ * (1 .. 10^9 ns).  The wait runs out, sets MOE_STATUS_TIMEOUT in *status and
+ * returns; the kernels of the library wait with these routines (200 ms limit).
+ * Nothing traps or stays in flight.  flag may be NULL for which = 0.
+ */
+MOE_API int moe_selftest_wait_timeout(int which, unsigned long long limit_ns, int32_t *status, uint32_t *flag,
+                                      void *stream);
+
+/*
  * Number of kernels moe_dispatch_layout (and moe_dispatch_layout_static)
  * launches for these sizes on the current device: 1 (single-launch layouts:
  * a thread-block cluster for up to 32768 pairs and E <= 512, else a cooperative grid when

@@ -57,6 +57,10 @@ def test_host_only_queries(lib):
     assert lib.moe_dispatch_layout_workspace(4096, 256, 8) >= 256 + 16 * 256 * 4
     assert lib.moe_dispatch_layout_workspace(4096, 2000, 8) == 0  # E > MOE_MAX_EXPERTS
     assert lib.moe_error_string(1) == b"invalid argument"
+    # the wait self-test refuses bad arguments before launching anything
+    assert lib.moe_selftest_wait_timeout(2, 1000, FAKE, FAKE, None) == 1
+    assert lib.moe_selftest_wait_timeout(0, 0, FAKE, None, None) == 1
+    assert lib.moe_selftest_wait_timeout(1, 1000, FAKE, None, None) == 1
     # invalid sizes answer 0 before any CUDA call
     assert lib.moe_dispatch_layout_kernels(0, 8, 2) == 0
     assert lib.moe_dispatch_layout_kernels(16, 2000, 2) == 0

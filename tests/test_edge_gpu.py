@@ -290,6 +290,31 @@ def test_fp8_dispatch_row_shapes(H, K):
     assert np.all(host(xd.view(torch.uint8))[~used] == 0x5A) and np.all(host(xs)[~used] == -7.0)
 
 
+@pytest.mark.parametrize("which", [0, 1])
+def test_bounded_wait_runs_out_and_reports(which):
+    """A wait that nothing completes (an mbarrier phase with no arrival, or a flag nobody
+    writes) gives up after its limit, reports MOE_STATUS_TIMEOUT, and the context stays
+    usable: a routing pass right after it matches the oracle."""
+    import time
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    B.moe_selftest_wait_timeout(which, 2_000_000, status, flag)  # 2 ms
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert status.item() == B.MOE_STATUS_TIMEOUT
+    w = synth.WORKLOADS["1"]
+    logits = synth.logits(w)
+    idx, _ = B.moe_route_topk(dev(logits), w.K)
+    lay = B.moe_dispatch_layout(idx, w.E, w.R, w.P)
+    ref_idx, _ = oracle.route_topk(logits, w.K)
+    np.testing.assert_array_equal(host(idx), ref_idx)
+    np.testing.assert_array_equal(host(lay.slot_of), oracle.layout(ref_idx, w.E, w.R, w.P)["slot_of"])
+    with pytest.raises(B.MoeError):
+        B.moe_selftest_wait_timeout(2, 1000, status)
+
+
 def test_fp8_dispatch_scale_rows_not_16_byte_aligned():
     """A scale array whose base is only 4-byte aligned: scales are stored per block."""
     rng = np.random.default_rng(5)
