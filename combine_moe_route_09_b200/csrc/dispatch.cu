@@ -171,6 +171,7 @@ constexpr int DQ_HDR = 128;                                  // per-stage header
 #define MOE_DQ_OUT_BUFS 2
 #endif
 constexpr int DQ_OUT_BUFS = MOE_DQ_OUT_BUFS;                 // bulk-store path: output staging buffers
+constexpr int DQ_BULK_MIN_ITEMS_PER_SM = 16;                 // bulk-store path from this many items per SM
 
 struct Fp8Args {
     const uint8_t *x;
@@ -519,9 +520,17 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
     if (a.stages < 3) a.stages = 3;
     a.obuf = a.bpc * 128 + (a.bpc * 4 + 15) / 16 * 16;
     a.scale_bulk = (blocks % 4 == 0 && a.bpc % 4 == 0 && (reinterpret_cast<uintptr_t>(xs) & 15) == 0) ? 1 : 0;
-    const bool bulk = MOE_DQ_BULK != 0;
-    const size_t smem = (size_t)a.stages * a.stage + (bulk ? (size_t)DQ_OUT_BUFS * a.obuf : 0) + 2 * DQ_MAX_STAGES * 8;
     const long long nitems = (long long)S * a.nchunks;
+    // Bulk stores from a staging buffer pay off once each CTA has several items
+    // to pipeline (prefill: 8192 items); with less than one item per CTA
+    // (decode: 256) the staging and its barriers only add latency, and
+    // per-thread stores are faster.
+    int dev = 0, sm_count = 0;
+    cudaError_t ae = cudaGetDevice(&dev);
+    if (ae == cudaSuccess) ae = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (ae != cudaSuccess) return ae;
+    const bool bulk = MOE_DQ_BULK != 0 && nitems >= (long long)DQ_BULK_MIN_ITEMS_PER_SM * sm_count;
+    const size_t smem = (size_t)a.stages * a.stage + (bulk ? (size_t)DQ_OUT_BUFS * a.obuf : 0) + 2 * DQ_MAX_STAGES * 8;
     auto go = [&](auto kern) -> cudaError_t {
         static KernelSlots<decltype(kern)> slots;
         unsigned grid = 1;
@@ -529,10 +538,12 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3(grid), dim3(DQ_THREADS), smem, st, a);
     };
-    constexpr bool BK = MOE_DQ_BULK != 0;
-    if (dtype == MOE_DTYPE_BF16)
-        return K == 8 ? go(&dispatch_fp8_kernel<false, 8, BK>) : go(&dispatch_fp8_kernel<false, 0, BK>);
-    return K == 8 ? go(&dispatch_fp8_kernel<true, 8, BK>) : go(&dispatch_fp8_kernel<true, 0, BK>);
+    if (dtype == MOE_DTYPE_BF16) {
+        if (bulk) return K == 8 ? go(&dispatch_fp8_kernel<false, 8, true>) : go(&dispatch_fp8_kernel<false, 0, true>);
+        return K == 8 ? go(&dispatch_fp8_kernel<false, 8, false>) : go(&dispatch_fp8_kernel<false, 0, false>);
+    }
+    if (bulk) return K == 8 ? go(&dispatch_fp8_kernel<true, 8, true>) : go(&dispatch_fp8_kernel<true, 0, true>);
+    return K == 8 ? go(&dispatch_fp8_kernel<true, 8, false>) : go(&dispatch_fp8_kernel<true, 0, false>);
 }
 
 }  // namespace moe

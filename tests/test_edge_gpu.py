@@ -269,13 +269,17 @@ def _midpoint_blocks(rng, S, H, in_bf16: bool):
     return synth.f32_to_bf16_bits(x) if in_bf16 else x
 
 
-@pytest.mark.parametrize("H,K", [(640, 8), (1664, 3), (4224, 8), (7296, 8), (7168, 5), (512, 32)])
-def test_fp8_dispatch_row_shapes(H, K):
+@pytest.mark.parametrize("S,H,K", [
+    # few items: per-thread stores
+    (300, 640, 8), (300, 1664, 3), (300, 4224, 8), (300, 7296, 8), (300, 7168, 5), (300, 512, 32),
+    # enough items per SM for the bulk-store path
+    (2400, 640, 8), (2400, 1664, 3), (1300, 7296, 8), (1200, 7168, 5), (2400, 512, 32),
+])
+def test_fp8_dispatch_row_shapes(S, H, K):
     """Rows whose block count is or is not a multiple of 4 (scale segments sent as one
-    bulk store per copy, or stored per block), one or two items per row, small and large K;
-    slots scattered over a larger capacity with unused rows left untouched."""
-    rng = np.random.default_rng(H + K)
-    S = 300
+    bulk store per copy, or stored per block), one or two items per row, small and large K,
+    on both store paths; slots scattered over a larger capacity with unused rows left untouched."""
+    rng = np.random.default_rng(H + K + S)
     cap = S * K + 77
     x = synth.f32_to_bf16_bits((rng.standard_normal((S, H)) * rng.uniform(0.01, 50, (S, 1))).astype(np.float32))
     slot = rng.permutation(cap)[:S * K].astype(np.int32).reshape(S, K)
@@ -315,10 +319,12 @@ def test_bounded_wait_runs_out_and_reports(which):
         B.moe_selftest_wait_timeout(2, 1000, status)
 
 
-def test_fp8_dispatch_scale_rows_not_16_byte_aligned():
-    """A scale array whose base is only 4-byte aligned: scales are stored per block."""
+@pytest.mark.parametrize("S", [64, 2400])
+def test_fp8_dispatch_scale_rows_not_16_byte_aligned(S):
+    """A scale array whose base is only 4-byte aligned: scales are stored per block
+    (on both store paths)."""
     rng = np.random.default_rng(5)
-    S, H, K = 64, 2048, 4
+    H, K = 2048, 4
     cap = S * K
     x = synth.f32_to_bf16_bits(rng.standard_normal((S, H)).astype(np.float32))
     slot = rng.permutation(cap).astype(np.int32).reshape(S, K)
