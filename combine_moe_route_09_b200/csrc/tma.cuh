@@ -162,10 +162,6 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 // Whole-CTA cluster barrier halves: every thread of every CTA of the cluster
 // arrives (release) and waits (acquire), from convergent code.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-// Arrival without release semantics: for a CTA that only signals "done reading".
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 // The shared::cluster address of `saddr` (a shared::cta address) in CTA `rank`.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
@@ -173,13 +169,9 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
+// Store into another CTA's shared memory (an address from cluster_map).
 __device__ __forceinline__ void st_cluster_s32(uint32_t addr, int v) {
     asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
 }
 
 }  // namespace moe
