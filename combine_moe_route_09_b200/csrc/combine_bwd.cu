@@ -24,13 +24,19 @@
 
 namespace moe {
 
-constexpr int BW_STAGES = 4;
+#ifndef MOE_BW_STAGES
+#define MOE_BW_STAGES 4
+#endif
+#ifndef MOE_BW_SMEM_BUDGET
+#define MOE_BW_SMEM_BUDGET (100 * 1024)
+#endif
+constexpr int BW_STAGES = MOE_BW_STAGES;
 constexpr int BW_CONSUMER_WARPS = 4;
 constexpr int BW_CONSUMERS = BW_CONSUMER_WARPS * 32;
 constexpr int BW_THREADS = BW_CONSUMERS + 32;
 constexpr int BW_MAX_CHUNK = BW_CONSUMERS * 16;
 constexpr int BW_HDR = 384;  // per stage: valid mask, the token's K weights (at 4), K slots (at 132)
-constexpr int BW_SMEM_BUDGET = 100 * 1024;
+constexpr int BW_SMEM_BUDGET = MOE_BW_SMEM_BUDGET;
 
 struct CombineBwdArgs {
     const uint8_t *g, *gn, *y;
