@@ -11,7 +11,7 @@
 //
 // Persistent kernel on the same pipeline as the forward combine: a producer
 // warp bulk-loads, per (token, chunk) item, the K gathered y chunks, the g
-// chunk and the gn chunk into a 3-stage ring (cp.async.bulk, mbarriers, no
+// chunk and the gn chunk into a 2-stage ring (cp.async.bulk, mbarriers, no
 // multicast); 4 consumer warps hold one 16-byte unit per thread.  Each CTA
 // takes whole tokens, so grad_w needs no atomics: per item every warp reduces
 // its dot-product partials with a fixed xor tree and lane k keeps pair k's
@@ -25,7 +25,7 @@
 namespace moe {
 
 #ifndef MOE_BW_STAGES
-#define MOE_BW_STAGES 3
+#define MOE_BW_STAGES 2
 #endif
 #ifndef MOE_BW_SMEM_BUDGET
 #define MOE_BW_SMEM_BUDGET (100 * 1024)
