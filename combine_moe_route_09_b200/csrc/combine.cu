@@ -29,11 +29,10 @@
 
 namespace moe {
 
-// Ring depth, chosen per launch (at most CB_MAX_STAGES): 3 stages when the
-// shared and residual rows ride along (3 CTAs per SM: 183.9 against 185.4 us per
-// DeepSeek-V3-shaped prefill step with 4), 4 otherwise (the plain and
-// unit-weight combines measured faster with 4).
-constexpr int CB_MAX_STAGES = 4;
+#ifndef MOE_CB_STAGES
+#define MOE_CB_STAGES 4
+#endif
+constexpr int CB_STAGES = MOE_CB_STAGES;
 constexpr int CB_CONSUMER_WARPS = 4;
 constexpr int CB_CONSUMERS = CB_CONSUMER_WARPS * 32;
 constexpr int CB_THREADS = CB_CONSUMERS + 32;
@@ -83,7 +82,6 @@ struct CombineArgs {
     int row_bytes;  // H * element size, a multiple of 16
     int chunk;      // bytes per work item, a multiple of 16, <= CB_MAX_CHUNK
     int nchunks;    // ceil(row_bytes / chunk)
-    int stages;     // ring depth (<= CB_MAX_STAGES)
 };
 
 constexpr int CB_HDR = 256;  // per-stage header: valid mask, then the token's K weights
@@ -95,17 +93,17 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
     extern __shared__ __align__(128) uint8_t smem[];
     // [STAGES][header | (K + 2) chunks: K gathered rows, shared_out, residual], then
     // the full / empty mbarriers of every stage
-    const int K = a.K, chunk = a.chunk, NS = a.stages;
+    const int K = a.K, chunk = a.chunk;
     const int stage_bytes = CB_HDR + (K + 2) * chunk;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * stage_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + CB_STAGES * stage_bytes);
     const uint32_t smem0 = smem_addr(smem);
     const uint32_t bar0 = smem_addr(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (CB_STAGES + s); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < CB_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), CB_CONSUMER_WARPS);
         }
@@ -135,7 +133,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
         bool ok = true;
         int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
         for (long long item = first; item < last && ok; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
-            const int s = i % NS;
+            const int s = i % CB_STAGES;
             if (t != t_cur) {
                 t_cur = t;
                 cur = nxt;
@@ -151,8 +149,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
                     nxt_w = a.topk_w ? __ldg(a.topk_w + (size_t)tn * K + lane) : 1.0f;
                 }
             }
-            if (i >= NS)
-                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / NS) - 1) & 1, a.status));
+            if (i >= CB_STAGES)
+                ok = __all_sync(FULL, mbar_wait(empty_bar(s), ((i / CB_STAGES) - 1) & 1, a.status));
             if (!ok) break;
             const int off = c * chunk;
             const uint32_t bytes = (uint32_t)min(chunk, a.row_bytes - off);
@@ -177,8 +175,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
         }
         // Never leave copies in flight: wait (bounded) for every stage still loading.
         if (lane == 0) {
-            for (int j = i - NS; j < i; ++j)
-                if (j >= 0) mbar_wait(full_bar(j % NS), (j / NS) & 1, a.status);
+            for (int j = i - CB_STAGES; j < i; ++j)
+                if (j >= 0) mbar_wait(full_bar(j % CB_STAGES), (j / CB_STAGES) & 1, a.status);
         }
         return;
     }
@@ -187,8 +185,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
     int i = 0;
     int t = (int)(first / a.nchunks), c = (int)(first - (long long)t * a.nchunks);
     for (long long item = first; item < last; ++item, ++i, (++c == a.nchunks ? (c = 0, ++t) : 0)) {
-        const int s = i % NS;
-        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / NS) & 1, a.status))) break;
+        const int s = i % CB_STAGES;
+        if (!__all_sync(FULL, mbar_wait(full_bar(s), (i / CB_STAGES) & 1, a.status))) break;
         const int off = c * chunk;
         const int bytes = min(chunk, a.row_bytes - off);
         const uint32_t stage = smem0 + (uint32_t)(s * stage_bytes);
@@ -234,18 +232,18 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
 
 static int combine_chunk(int K, int row_bytes) {
     int chunk = CB_MAX_CHUNK;
-    while (chunk > 256 && CB_MAX_STAGES * (CB_HDR + (K + 2) * chunk) > CB_SMEM_BUDGET) chunk >>= 1;
+    while (chunk > 256 && CB_STAGES * (CB_HDR + (K + 2) * chunk) > CB_SMEM_BUDGET) chunk >>= 1;
     return chunk < row_bytes ? chunk : row_bytes;
 }
 
-static size_t combine_smem(int K, int chunk, int stages) {
-    return (size_t)stages * (CB_HDR + (K + 2) * chunk) + 2 * stages * 8;
+static size_t combine_smem(int K, int chunk) {
+    return (size_t)CB_STAGES * (CB_HDR + (K + 2) * chunk) + 2 * CB_STAGES * 8;
 }
 
 template <bool F32, bool SH, bool RS, bool RNR>
 static cudaError_t launch_cb(const CombineArgs &a, cudaStream_t st) {
     auto kern = combine_kernel<F32, SH, RS, RNR>;
-    const size_t smem = combine_smem(a.K, a.chunk, a.stages);
+    const size_t smem = combine_smem(a.K, a.chunk);
     static KernelSlots<decltype(kern)> slots;
     int sms = 0, per_sm = 0;
     cudaError_t e = slots.prepare(kern, CB_THREADS, smem, &sms, &per_sm);
@@ -287,7 +285,6 @@ cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_
     a.row_bytes = H * (f32 ? 4 : 2);
     a.chunk = combine_chunk(K, a.row_bytes);
     a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
-    a.stages = (shared_out && residual) ? 3 : CB_MAX_STAGES;
     return f32 ? launch_cb_dt<true>(a, st) : launch_cb_dt<false>(a, st);
 }
 
