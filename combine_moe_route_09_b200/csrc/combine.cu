@@ -29,10 +29,7 @@
 
 namespace moe {
 
-#ifndef MOE_CB_STAGES
-#define MOE_CB_STAGES 4
-#endif
-constexpr int CB_STAGES = MOE_CB_STAGES;
+constexpr int CB_STAGES = 4;
 constexpr int CB_CONSUMER_WARPS = 4;
 constexpr int CB_CONSUMERS = CB_CONSUMER_WARPS * 32;
 constexpr int CB_THREADS = CB_CONSUMERS + 32;
