@@ -597,53 +597,47 @@ __global__ void __launch_bounds__(LC_THREADS)
     }
     if (bad) set_status(status, MOE_STATUS_BAD_INDEX);
     __syncthreads();
-    // tpe consecutive lanes share an expert, each covering LC_WARPS / tpe warps
+    // per-warp counts -> exclusive prefix over warps, and the tile's total per
+    // expert: tpe consecutive lanes share an expert, each summing LC_WARPS / tpe
+    // warps, then an exclusive scan across those lanes (shuffles)
     int tpe = 1;
     while (tpe < 32 && tpe < LC_WARPS && tpe * 2 * E <= LC_THREADS) tpe *= 2;
-    const int wpt = LC_WARPS / tpe, sub = lane & (tpe - 1), epw = 32 / tpe;
-    const int w0 = sub * wpt;
-    // the tile's count per expert (a sum over the warps' counts) ...
-    for (int e0 = w * epw; e0 < E; e0 += LC_WARPS * epw) {  // warp-uniform trip count
-        const int e = e0 + lane / tpe;
-        const bool ok = e < E;
-        int part = 0;
-        if (ok)
-            for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * WS + e];
-        for (int off = 1; off < tpe; off <<= 1) part += __shfl_xor_sync(FULL, part, off, tpe);
-        if (ok && sub == 0) thist[e] = part;
+    {
+        const int wpt = LC_WARPS / tpe, sub = lane & (tpe - 1), epw = 32 / tpe;
+        const int w0 = sub * wpt;
+        for (int e0 = w * epw; e0 < E; e0 += LC_WARPS * epw) {  // warp-uniform trip count
+            const int e = e0 + lane / tpe;
+            const bool ok = e < E;
+            int part = 0;
+            if (ok)
+                for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * WS + e];
+            int incl = part;  // inclusive scan over the tpe lanes of this expert
+            for (int off = 1; off < tpe; off <<= 1) {
+                const int o = __shfl_up_sync(FULL, incl, off, tpe);
+                if (sub >= off) incl += o;
+            }
+            if (ok) {
+                int run = incl - part;
+                for (int ww = w0; ww < w0 + wpt; ++ww) {
+                    const int c = whist[ww * WS + e];
+                    whist[ww * WS + e] = (uint16_t)run;
+                    run += c;
+                }
+                if (sub == tpe - 1) thist[e] = incl;
+            }
+        }
     }
     __syncthreads();
-    // ... pushed into row `me` of every CTA's allh (stores into the cluster's
-    // distributed shared memory) before the one cluster barrier: after it every
-    // CTA holds all tiles' counts locally, and no CTA touches another's shared
-    // memory again, so none has to wait for the others before exiting
+    // push this tile's counts into row `me` of every CTA's allh (stores into the
+    // cluster's distributed shared memory), then one cluster barrier: after it
+    // every CTA holds all tiles' counts locally, and no CTA touches another's
+    // shared memory again, so none has to wait for the others before exiting
     const uint32_t ah = smem_addr(allh) + 4u * me * (uint32_t)E;
     for (int idx = tid; idx < C * E; idx += LC_THREADS) {
         const int c = idx / E, e = idx - c * E;
         st_cluster_s32(cluster_map(ah + 4u * e, (uint32_t)c), thist[e]);
     }
     cluster_arrive();
-    // while the other CTAs arrive: per-warp counts -> exclusive prefix over warps
-    for (int e0 = w * epw; e0 < E; e0 += LC_WARPS * epw) {  // warp-uniform trip count
-        const int e = e0 + lane / tpe;
-        const bool ok = e < E;
-        int part = 0;
-        if (ok)
-            for (int ww = w0; ww < w0 + wpt; ++ww) part += whist[ww * WS + e];
-        int incl = part;  // inclusive scan over the tpe lanes of this expert
-        for (int off = 1; off < tpe; off <<= 1) {
-            const int o = __shfl_up_sync(FULL, incl, off, tpe);
-            if (sub >= off) incl += o;
-        }
-        if (ok) {
-            int run = incl - part;
-            for (int ww = w0; ww < w0 + wpt; ++ww) {
-                const int c = whist[ww * WS + e];
-                whist[ww * WS + e] = (uint16_t)run;
-                run += c;
-            }
-        }
-    }
     cluster_wait();
 
     // ---- totals and the count of the tiles below this one ----
