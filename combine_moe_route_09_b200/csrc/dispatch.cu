@@ -24,14 +24,16 @@
 //    quantise: each thread owns 16 channels, the 8 threads of a 128-channel
 //    block reduce amax with xor-shuffles, s = amax / 448 (IEEE division) and
 //    q = e4m3(x / s) with the quotient correctly rounded (Markstein's
-//    correction of x * RN(1/s); plain IEEE division for subnormal s) and
-//    cvt.rn.satfinite.e4m3x2.  The quantised item (codes, then its block
-//    scales) is staged in one of DQ_OUT_BUFS shared-memory buffers, and after a named
-//    barrier one thread sends the K copies as TMA bulk stores (one per copy
-//    for the codes, one for the scales when the segment is whole 16-byte
-//    units, else the blocks' lead threads store the scales).  Whole-row bulk
-//    stores write the scattered destination rows faster than per-thread
-//    16-byte stores.
+//    correction of x * RN(1/s); plain IEEE division for s < 2^-90) and
+//    cvt.rn.satfinite.e4m3x2.  With at least DQ_BULK_MIN_ITEMS_PER_SM items
+//    per SM the quantised item (codes, then its block scales) is staged in
+//    one of DQ_OUT_BUFS shared-memory buffers, and after a named barrier one
+//    thread sends the K copies as TMA bulk stores (one per copy for the
+//    codes, one for the scales when the segment is whole 16-byte units, else
+//    the blocks' lead threads store the scales): whole-item bulk stores write
+//    the scattered destination rows faster.  With fewer items (decode sizes)
+//    each thread stores its codes K times from registers, which is faster
+//    when the staging cannot be amortised.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tma.cuh"
