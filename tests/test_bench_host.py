@@ -100,3 +100,26 @@ def test_algorithmic_bytes_formula():
     assert b["dispatch"] == S * H * 2 + S * K * H + S * K * (H // 128) * 4 + S * K * 4
     assert b["combine"] == S * K * H * 2 + S * K * 8 + 4 * S * H * 2
     assert round(b["dispatch"] / 1e6, 1) == 301.1 and round(b["combine"] / 1e6, 1) == 704.9
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic is read from a profile summary only while the kernel
+    source it was captured from is unchanged (same SHA-256) and the workload matches."""
+    import hashlib
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = tmp_path / "combine_moe_route_09_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k.cu").write_text("// kernel v1\n")
+    sha = hashlib.sha256(b"// kernel v1\n").hexdigest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "k_w.md").write_text(f"# k\n\nkernel_source_sha256: {sha}\nworkload: w\ndram_bytes_per_launch: 12345\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k.cu", "w") == 12345
+    assert bench.recorded_traffic("k.cu", "other") is None
+    (src / "k.cu").write_text("// kernel v2\n")
+    assert bench.recorded_traffic("k.cu", "w") is None
+    assert bench.recorded_traffic("missing.cu", "w") is None
