@@ -53,7 +53,8 @@ def algorithmic_bytes(w) -> dict:
     if w.quant == "fp8":
         dispatch += S * K * (H // 128) * 4
     combine = S * K * H * b + S * K * 8 + (4 * S * H * b if w.fused else S * H * b)
-    return dict(route=route, layout=layout, dispatch=dispatch, combine=combine)
+    return dict(route=route, layout=layout, dispatch=dispatch, combine=combine,
+                route_dispatch=route + layout + dispatch)
 
 
 def workload_config(w, world: int) -> dict:
@@ -192,31 +193,80 @@ def barrier(world: int):
 # CPU oracle baseline (test infrastructure; this leg alone may run it)
 # ----------------------------------------------------------------------------------------------
 
-def oracle_pass(w, inp: dict, S: int):
+def oracle_pass(w, inp: dict, S: int, threads: int = 1):
+    """One routing pass of the first S tokens through the oracle.
+
+    With threads > 1 the per-token steps (route, dispatch, combine) are split
+    over contiguous token ranges, one range per thread (the oracle's C calls
+    release the GIL); the layout, a global counting sort, runs once."""
+    import numpy as np
+
     import oracle
 
     lg = inp["logits"][:S]
-    idx, wt = oracle.route_topk(lg, w.K)
-    lay = oracle.layout(idx, w.E, w.R, w.P)
+    bounds = [S * i // threads for i in range(threads + 1)]
+    ranges = [(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
     q = oracle.QUANT_FP8_E4M3_B128 if w.quant == "fp8" else oracle.QUANT_NONE
-    oracle.dispatch(inp["x"][:S], lay["slot_of"], lay["cap"], quant=q)
-    y = inp["y"][:lay["cap"]]
-    oracle.combine(y, lay["slot_of"], wt, inp["shared"][:S] if w.fused else None,
-                   inp["residual"][:S] if w.fused else None)
+
+    def par(fn):
+        if len(ranges) == 1:
+            return [fn(*ranges[0])]
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=len(ranges)) as ex:
+            return list(ex.map(lambda r: fn(*r), ranges))
+
+    parts = par(lambda a, b: oracle.route_topk(lg[a:b], w.K))
+    idx = np.concatenate([p[0] for p in parts])
+    wt = np.concatenate([p[1] for p in parts])
+    lay = oracle.layout(idx, w.E, w.R, w.P)
+    cap, H = lay["cap"], w.H
+    x = inp["x"][:S]
+    if q == oracle.QUANT_FP8_E4M3_B128:
+        xd, xs = np.zeros((cap, H), np.uint8), np.zeros((cap, H // 128), np.float32)
+    else:
+        xd, xs = np.zeros((cap, H), x.dtype), None
+    par(lambda a, b: oracle.dispatch(x[a:b], lay["slot_of"][a:b], cap, quant=q, xd=xd, xs=xs))
+    y = inp["y"][:cap]
+    sh = inp["shared"][:S] if w.fused else None
+    rs = inp["residual"][:S] if w.fused else None
+    outs = par(lambda a, b: oracle.combine(y, lay["slot_of"][a:b], wt[a:b], None if sh is None else sh[a:b],
+                                           None if rs is None else rs[a:b]))
+    out = np.concatenate([o[0] for o in outs])
+    rnr = np.concatenate([o[1] for o in outs]) if outs[0][1] is not None else None
+    return dict(topk_idx=idx, topk_w=wt, layout=lay, xd=xd, xs=xs, out=out, out_no_routed=rnr)
 
 
-def cpu_baseline(w, inp: dict, min_seconds: float = 10.0) -> dict:
-    """Full workload through the oracle, repeated until min_seconds of CPU work."""
-    n, t0 = 0, time.perf_counter()
-    while True:
-        oracle_pass(w, inp, w.S)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= min_seconds:
-            break
-    return {"value": w.S * n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} full pass(es) of {w.name} (S={w.S}) through the single-threaded C oracle, "
-                      f"{el:.1f} s"}
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def _time_passes(w, inp, S, threads, min_passes, min_seconds):
+    times = []
+    t_all = time.perf_counter()
+    while len(times) < min_passes or time.perf_counter() - t_all < min_seconds:
+        t0 = time.perf_counter()
+        oracle_pass(w, inp, S, threads)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def cpu_baseline(w, inp: dict) -> dict:
+    """The oracle on this machine's host cores over full passes of the workload:
+    single-threaded, and split over token ranges on every core this process may
+    use; each the median of at least 3 passes."""
+    n = host_threads()
+    single = _time_passes(w, inp, w.S, 1, 3, 0.0)
+    multi = _time_passes(w, inp, w.S, n, 3, 5.0)
+    med1, medn = statistics.median(single), statistics.median(multi)
+    return {"value": w.S / medn, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "sample": f"median of {len(multi)} full passes of {w.name} (S={w.S}) through the C oracle, "
+                      f"per-token steps split over {n} threads by token range",
+            "host_cpu_count": os.cpu_count(), "threads": n,
+            "single_thread": {"value": w.S / med1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"median of {len(single)} full passes, one thread"}}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -233,44 +283,177 @@ def host_inputs(w) -> dict:
 
 
 def run_reference(args, w, world):
-    """CPU oracle as the reference arm: rank 0 only, a bounded token sample per step."""
+    """CPU oracle as the reference arm: rank 0 only, every host core, a bounded
+    token sample per step."""
     inp = host_inputs(w)
-    n_cal = min(w.S, 256)
+    n = host_threads()
+    n_cal = min(w.S, max(256, 64 * n))
     t0 = time.perf_counter()
-    oracle_pass(w, inp, n_cal)
+    oracle_pass(w, inp, n_cal, n)
     per_tok = (time.perf_counter() - t0) / n_cal
     budget = 60.0  # seconds for warm-up + timed steps together
     S_sample = int(max(1, min(w.S, budget / max(1, args.steps + args.warmup) / per_tok)))
     for _ in range(args.warmup):
-        oracle_pass(w, inp, S_sample)
+        oracle_pass(w, inp, S_sample, n)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_pass(w, inp, S_sample)
+        oracle_pass(w, inp, S_sample, n)
     el = time.perf_counter() - t0
     value = S_sample * args.steps / el
     sample = (f"first {S_sample} of {w.S} tokens of {w.name} per step (same H, E, K, R, padding, "
-              f"quantisation and epilogue), single-threaded C oracle")
+              f"quantisation and epilogue), C oracle split over {n} threads by token range")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded)", "config": workload_config(w, world),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": 1,
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": n,
+                         "host_cpu_count": os.cpu_count(), "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, w, rank, world, local_rank):
+def _pct(v, q):
+    v = sorted(v)
+    if not v:
+        return None
+    i = (len(v) - 1) * q
+    lo, hi = int(i), min(int(i) + 1, len(v) - 1)
+    return v[lo] + (v[hi] - v[lo]) * (i - lo)
+
+
+def _stats(v):
+    return {"median": statistics.median(v), "p10": _pct(v, 0.1), "p90": _pct(v, 0.9), "n": len(v)}
+
+
+def _graph_of(calls, n):
+    """CUDA graph of n repetitions of the calls, captured on a side stream."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            for c in calls:
+                c()
+    return g
+
+
+def time_windows(step, K, windows, world, device):
+    """`windows` windows of exactly K steps each, every window bracketed by a
+    barrier and a device synchronisation on both sides; ms per window (max over ranks)."""
+    import torch
+
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for _ in range(windows):
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(K):
+            step()
+        b.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        out.append(max_over_ranks(a.elapsed_time(b), world, device))
+    return out
+
+
+def phases_in_graph(phases, steps, windows):
+    """Per-phase device time inside a CUDA graph of `steps` steps: an event node
+    (cudaEventRecordExternal) before the first phase and after each phase of
+    every step.  The event nodes sit between the kernels, so no phase overlaps
+    its neighbour here; returns µs samples per phase."""
+    import torch
+
+    n = len(phases)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)] for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            evs[i][0].record()
+            for j, (_, call) in enumerate(phases):
+                call()
+                evs[i][j + 1].record()
+    g.replay()
+    torch.cuda.synchronize()
+    samples = {name: [] for name, _ in phases}
+    for _ in range(windows):
+        g.replay()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            for j, (name, _) in enumerate(phases):
+                samples[name].append(evs[i][j].elapsed_time(evs[i][j + 1]) * 1e3)
+    del g
+    return samples
+
+
+def phases_marginal(phases, steps, windows):
+    """Marginal cost of each phase in the graph-replayed step: the time per step
+    of a graph of the first j+1 phases minus that of the first j phases (every
+    graph `steps` steps long, consecutive kernels overlapping through
+    programmatic dependent launch as in the product step).  The marginal costs
+    add up to the step time; returns µs per phase."""
+    import torch
+
+    per_prefix = []
+    for j in range(len(phases)):
+        g = _graph_of([c for _, c in phases[:j + 1]], steps)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(windows):
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / steps)
+        del g
+        per_prefix.append(statistics.median(ts))
+    out, prev = {}, 0.0
+    for (name, _), t in zip(phases, per_prefix):
+        out[name] = t - prev
+        prev = t
+    return out
+
+
+def phases_eager(phases, steps):
+    """Eager calls with an event between consecutive kernels (NVTX range per phase)."""
+    import torch
+
+    n = len(phases)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record()
+        for j, (name, call) in enumerate(phases):
+            with torch.cuda.nvtx.range(name):
+                call()
+            ev[i][j + 1].record()
+    torch.cuda.synchronize()
+    return {name: [ev[i][j].elapsed_time(ev[i][j + 1]) * 1e3 for i in range(steps)]
+            for j, (name, _) in enumerate(phases)}
+
+
+def _phase_table(us: dict, ab: dict, peak: float) -> dict:
+    out = {}
+    for name, t in us.items():
+        gbs = ab[name] / (t * 1e-6) / 1e9
+        out[name] = {"us": t, "algorithmic_bytes": ab[name], "gb_s": gbs, "frac_of_peak": gbs / peak,
+                     "frac_of_nominal_8tbs": gbs / 8000.0}
+    return out
+
+
+def measure_workload(w, args, world, local_rank, device, windows, e2e: bool):
+    """Times one workload: the graph-replayed step over `windows` windows of K
+    steps, then its phases (event nodes in the graph, marginal costs, eager)."""
     import torch
 
     from combine_moe_route_09_b200 import synth
     from combine_moe_route_09_b200.buffer import MoeBuffer
 
-    torch.cuda.set_device(local_rank)
-    device = torch.device("cuda", local_rank)
     inp = host_inputs(w)
     pinned = {k: synth.to_torch(v).pin_memory() for k, v in inp.items()}
     d = {k: v.to(device, non_blocking=True) for k, v in pinned.items()}
@@ -278,13 +461,11 @@ def run_ours(args, w, rank, world, local_rank):
     buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device)
     sh, rs = (d["shared"], d["residual"]) if w.fused else (None, None)
     torch.cuda.synchronize()
-
     for _ in range(args.warmup):
         buf.step(d["logits"], d["x"], d["y"], sh, rs)
     torch.cuda.synchronize()
     if buf.read_status() != 0:
         raise RuntimeError("device status flagged a problem during warm-up")
-
     graph = None
     if args.graph:
         graph = buf.capture(d["logits"], d["x"], d["y"], sh, rs)
@@ -293,67 +474,30 @@ def run_ours(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
         if buf.read_status() != 0:
             raise RuntimeError("device status flagged a problem in the captured step")
+    step = graph.replay if graph is not None else (lambda: buf.step(d["logits"], d["x"], d["y"], sh, rs))
 
-    def one_step():
-        if graph is not None:
-            graph.replay()
-        else:
-            buf.step(d["logits"], d["x"], d["y"], sh, rs)
-
-    # ---- timed region 1 (value): K steps back to back, events only at the ends, so
-    # consecutive kernels overlap through programmatic dependent launch ----
     K = args.steps
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    barrier(world)
-    torch.cuda.synchronize()
-    t_start.record()
     h0 = time.perf_counter()
-    for _ in range(K):
-        one_step()
-    t_end.record()
-    host_us = (time.perf_counter() - h0) / K * 1e6
+    win_ms = time_windows(step, K, windows, world, device)
+    host_us = (time.perf_counter() - h0) / (K * windows) * 1e6
+    phases = buf.step_phases(d["logits"], d["x"], d["y"], sh, rs)
+    Kp = max(1, min(K, 50))
+    ev_nodes = phases_in_graph(phases, Kp, max(3, windows // 2))
+    marginal = phases_marginal(phases, Kp, max(3, windows // 2))
+    eager = phases_eager(phases, Kp)
     torch.cuda.synchronize()
-    barrier(world)
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, device)
-
-    # ---- timed region 2 (per kernel): the same K steps with an event between
-    # kernels, on the launching stream; these durations feed the roofline ----
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(K):
-        e = ev[i]
-        e[0].record()
-        buf.route(d["logits"])
-        e[1].record()
-        buf.plan()
-        e[2].record()
-        buf.dispatch(d["x"])
-        e[3].record()
-        buf.combine(d["y"], sh, rs)
-        e[4].record()
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = sampler.stop()
-    phase_names = ["route", "layout", "dispatch", "combine"]
-    phase_ms = {p: statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
-                for j, p in enumerate(phase_names)}
     status = buf.read_status()
     counts_ok = int(buf.layout.counts.sum().item()) == w.S * w.K
     if status != 0 or not counts_ok:
         raise RuntimeError(f"bench sanity check failed: status={status} counts_ok={counts_ok}")
 
-    # ---- end to end: pinned host inputs in, both residual streams out, every step ----
-    e2e = None
-    if not args.no_e2e:
+    e2e_res = None
+    if e2e:
         Ke = min(K, args.e2e_steps)
         out_h = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
         rnr_h = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory() if w.fused else None
         h2d = sum(v.numel() * v.element_size() for v in pinned.values())
         d2h = out_h.numel() * out_h.element_size() * (2 if w.fused else 1)
-
         # Inputs go in on the compute stream; each step's outputs come back on a copy
         # stream, so that read overlaps the next step's input copies (PCIe is full
         # duplex).  A step's kernels wait for the previous read of the outputs.
@@ -389,44 +533,95 @@ def run_ours(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
-        e2e = {"value": w.S * world * Ke / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
-               "ms_per_step": e2e_ms / Ke,
-               "path": "MoeBuffer.step via the C ABI; pinned host inputs copied in and both residual "
-                       "streams copied out each step (the copy out overlapping the next step's copy in), "
-                       "inside the timed region"}
+        e2e_res = {"value": w.S * world * Ke / (e2e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+                   "ms_per_step": e2e_ms / Ke,
+                   "path": "MoeBuffer.step via the C ABI; pinned host inputs copied in and both residual "
+                           "streams copied out each step (the copy out overlapping the next step's copy in), "
+                           "inside the timed region"}
 
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = read_peak_hbm()
+    per_step = [t / K for t in win_ms]
+    med = statistics.median(per_step)
+    ph_in = {k: statistics.median(v) for k, v in ev_nodes.items()}
+    res = {
+        "ms_per_step": med, "ms_per_step_stats": _stats(per_step), "windows": windows, "steps_per_window": K,
+        "tokens_per_s": w.S * world / (med * 1e-3),
+        "phases": _phase_table(ph_in, ab, peak),
+        "phases_p10_p90_us": {k: [_pct(v, 0.1), _pct(v, 0.9)] for k, v in ev_nodes.items()},
+        "phases_marginal": _phase_table(marginal, ab, peak),
+        "phases_eager": _phase_table({k: statistics.median(v) for k, v in eager.items()}, ab, peak),
+        "gpu_launches_per_step": buf.kernels_per_step,
+        "host_enqueue_us_per_step": host_us,
+        "graph": graph is not None,
+    }
+    res["_buf"], res["_inp"], res["_e2e"], res["_peak"] = buf, inp, e2e_res, (peak, peak_kind)
+    return res
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+
+    from combine_moe_route_09_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    windows = max(10, args.windows)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    head = measure_workload(w, args, world, local_rank, device, windows, e2e=not args.no_e2e)
+    others = {}
+    if not args.headline_only:
+        for key, ow in synth.WORKLOADS.items():
+            if ow.name == w.name:
+                continue
+            r = measure_workload(ow, args, world, local_rank, device, windows, e2e=False)
+            for k in ("_buf", "_inp", "_e2e", "_peak"):
+                r.pop(k)
+            r["config"] = {kk: vv for kk, vv in workload_config(ow, world).items() if kk != "l2"}
+            others[key] = r
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    buf, inp, e2e, (peak, peak_kind) = head.pop("_buf"), head.pop("_inp"), head.pop("_e2e"), head.pop("_peak")
     if rank != 0:
         return
     ab = algorithmic_bytes(w)
-    peak, peak_kind = read_peak_hbm()
-    phases = {}
-    for p in phase_names:
-        gbs = ab[p] / (phase_ms[p] * 1e-3) / 1e9
-        phases[p] = {"us": phase_ms[p] * 1e3, "algorithmic_bytes": ab[p], "gb_s": gbs,
-                     "frac_of_peak": gbs / peak}
-    dc_ms = phase_ms["dispatch"] + phase_ms["combine"]
-    dc_gbs = (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3) / 1e9
-    comb = phases["combine"]
+    ph = head["phases"]
+    dname = "route_dispatch" if "route_dispatch" in ph else "dispatch"
+    dc_us = ph[dname]["us"] + ph["combine"]["us"]
+    dc_gbs = (ab[dname] + ab["combine"]) / (dc_us * 1e-6) / 1e9
+    comb = ph["combine"]
     roofline = {"kernel": "combine_kernel (gather + weighted sum + dual residual)", "bound": "hbm",
                 "achieved": comb["gb_s"], "peak": peak, "unit": "GB/s", "frac": comb["gb_s"] / peak,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s",
                 "algorithmic_bytes_per_launch": ab["combine"],
+                "duration_us": comb["us"],
+                "timing": "CUDA event nodes around the kernel inside the graph-replayed step",
                 "traffic": recorded_traffic("combine.cu", w.name)}
+    K = args.steps
     line = {
-        "metric": METRIC, "value": w.S * world * K / (total_ms / 1e3), "unit": "tokens/s",
-        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "ms_per_step_stats": head["ms_per_step_stats"], "windows": head["windows"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; no dataset or weights)", "config": workload_config(w, world),
-        "dispatch_combine": {"tokens_per_s": w.S * world / (dc_ms * 1e-3), "effective_gb_s": dc_gbs,
+        "dispatch_combine": {"tokens_per_s": w.S * world / (dc_us * 1e-6), "effective_gb_s": dc_gbs,
                              "frac_of_peak": dc_gbs / peak, "frac_of_nominal_8tbs": dc_gbs / 8000.0},
-        "phases": phases, "roofline": roofline, "e2e": e2e,
-        "gpu_launches": K * buf.kernels_per_step, "clocks": clocks,
-        "timing": "value: K steps back to back (events at the ends only)"
-                  + (", each step one CUDA-graph replay" if graph is not None else ", eager calls")
-                  + "; phases/roofline: a second pass of K eager steps with an event between kernels",
-        "host_enqueue_us_per_step": host_us,
+        "phases": ph, "phases_p10_p90_us": head["phases_p10_p90_us"],
+        "phases_marginal": head["phases_marginal"], "phases_eager": head["phases_eager"],
+        "roofline": roofline, "e2e": e2e,
+        "gpu_launches": K * head["gpu_launches_per_step"], "clocks": clocks,
+        "timing": ("value: median over windows of exactly K steps (barrier + synchronize around each window), "
+                   + ("each step one CUDA-graph replay" if head["graph"] else "eager calls")
+                   + "; phases: CUDA event nodes between the kernels inside a graph of min(K, 50) steps; "
+                     "phases_marginal: leave-one-out graphs (a graph of the first j+1 phases minus one of the "
+                     "first j), consecutive kernels overlapping as in the step; phases_eager: eager calls with "
+                     "an event between kernels"),
+        "host_enqueue_us_per_step": head["host_enqueue_us_per_step"],
+        "workloads": others,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp)
@@ -690,6 +885,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--windows", type=int, default=10,
+                    help="timed windows of K steps each (at least 10); the value is their median")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other workloads (the JSON line's `workloads` object)")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time the value pass as CUDA-graph replays of one step (default; "
                          "--no-graph times eager calls)")

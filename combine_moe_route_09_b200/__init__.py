@@ -16,11 +16,19 @@ raises if it is missing.
 from .binding import (  # noqa: F401
     MOE_DTYPE_BF16,
     MOE_DTYPE_F32,
+    MOE_ERR_CUDA,
+    MOE_ERR_INVALID_ARG,
+    MOE_ERR_SCRATCH_TOO_SMALL,
+    MOE_MAX_EXPERTS,
+    MOE_MAX_TOPK,
+    MOE_OK,
     MOE_QUANT_FP8_E4M3_B128,
     MOE_QUANT_NONE,
+    MOE_STATIC_LAYOUT_SCRATCH_BYTES,
     MOE_STATUS_BAD_INDEX,
     MOE_STATUS_BAD_SLOT,
     MOE_STATUS_OVERFLOW,
+    MOE_STATUS_TIMEOUT,
     Layout,
     MoeError,
     lib,
@@ -32,9 +40,11 @@ from .binding import (  # noqa: F401
     moe_dispatch_backward,
     moe_dispatch_layout,
     moe_dispatch_layout_kernels,
+    moe_dispatch_layout_static,
     moe_dispatch_layout_workspace,
     moe_dispatch_route_weights,
-    moe_route_topk,
     moe_route_sigmoid_grouped,
+    moe_route_topk,
     moe_route_topk_backward,
+    moe_selftest_wait_timeout,
 )

@@ -132,12 +132,21 @@ class MoeBuffer:
             self._p_rnr if fused else None, self._p_status, self._stream(stream)))
         return self.out, (self.out_no_routed if fused else None)
 
+    def step_phases(self, logits, x, y, shared_out=None, residual=None, stream=None):
+        """The calls of one full pass, in order, as (phase name, zero-argument call)
+        pairs; running them in order is one step (y = expert outputs)."""
+        return [
+            ("route", lambda: self.route(logits, stream)),
+            ("layout", lambda: self.plan(stream=stream)),
+            ("dispatch", lambda: self.dispatch(x, stream)),
+            ("combine", lambda: self.combine(y, shared_out, residual, stream=stream)),
+        ]
+
     def step(self, logits, x, y, shared_out=None, residual=None, stream=None):
         """One full pass: route, layout, dispatch, combine (y = expert outputs)."""
-        self.route(logits, stream)
-        self.plan(stream=stream)
-        self.dispatch(x, stream)
-        return self.combine(y, shared_out, residual, stream=stream)
+        for _, call in self.step_phases(logits, x, y, shared_out, residual, stream):
+            call()
+        return self.out, (self.out_no_routed if (shared_out is not None and residual is not None) else None)
 
     def capture(self, logits, x, y, shared_out=None, residual=None):
         """Records one step into a CUDA graph and returns it (``graph.replay()``

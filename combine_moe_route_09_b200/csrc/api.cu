@@ -1,6 +1,12 @@
 // C-ABI entry points: host-side argument checks, then the launches.  Every
 // entry point only enqueues work on the caller's stream.
+//
+// Each entry point that enqueues GPU work opens an NVTX range named after it
+// for the time of the call, so a profiler's timeline labels the launches of
+// each step of the path.  NVTX is header-only here: with no tool attached the
+// range calls do nothing.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -19,6 +25,14 @@ int current_sms() {
 int esize(int dtype) { return dtype == MOE_DTYPE_F32 ? 4 : (dtype == MOE_DTYPE_BF16 ? 2 : 0); }
 
 int to_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// NVTX range for the lifetime of one entry-point call.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 
 // Activation rows: 16-byte aligned base and a row size that is a multiple of 16 bytes.
 bool rows_ok(const void *p, int H, int bytes_per_elem) {
@@ -53,6 +67,7 @@ int moe_route_topk(const float *logits, int S, int E, int K, int32_t *topk_idx, 
     if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_route_topk");
     return to_rc(moe::launch_route_topk(logits, S, E, K, topk_idx, topk_w,
                                         static_cast<cudaStream_t>(stream), current_sms()));
 }
@@ -61,6 +76,7 @@ int moe_selftest_wait_timeout(int which, unsigned long long limit_ns, int32_t *s
                               void *stream) {
     if ((which != 0 && which != 1) || limit_ns < 1 || limit_ns > 1000000000ull) return MOE_ERR_INVALID_ARG;
     if (!status || !aligned(status, 4) || (which == 1 && (!flag || !aligned(flag, 4)))) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_selftest_wait_timeout");
     return to_rc(moe::launch_wait_selftest(which, limit_ns, status, flag, static_cast<cudaStream_t>(stream)));
 }
 
@@ -77,6 +93,7 @@ int moe_dispatch_route_weights(const float *topk_w, const int32_t *row_src, int 
     if (!aligned(row_src, 4) || !aligned(route_weights, 4) || (topk_w && !aligned(topk_w, 4)) ||
         (status && !aligned(status, 4)))
         return MOE_ERR_INVALID_ARG;
+    const Range range("moe_dispatch_route_weights");
     return to_rc(moe::launch_route_weights(topk_w, row_src, (int64_t)S * K, cap, route_weights, status,
                                            static_cast<cudaStream_t>(stream), current_sms()));
 }
@@ -94,6 +111,7 @@ int moe_route_sigmoid_grouped(const float *logits, const float *bias, int S, int
     if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || (bias && !aligned(bias, 4)))
         return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_route_sigmoid_grouped");
     return to_rc(moe::launch_route_sigmoid_grouped(logits, bias, S, E, K, n_group, n_group > 1 ? topk_group : 1,
                                                    normalize, scale, topk_idx, topk_w,
                                                    static_cast<cudaStream_t>(stream), current_sms()));
@@ -123,6 +141,7 @@ int moe_dispatch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int
     const void *ptrs[] = {topk_idx, counts, offsets, rank_offsets, slot_of, row_src, status};
     for (const void *p : ptrs)
         if (p && !aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_dispatch_layout");
     return to_rc(moe::launch_layout(topk_idx, S, E, K, R, token_padding, counts, offsets,
                                     rank_offsets, slot_of, row_src, cap, workspace, status,
                                     static_cast<cudaStream_t>(stream)));
@@ -144,6 +163,7 @@ int moe_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *s
             return MOE_ERR_INVALID_ARG;
     }
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_dispatch");
     return to_rc(moe::launch_dispatch(x, dtype, S, H, K, slot_of, quant, xd, xs, cap, status,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -164,6 +184,7 @@ int moe_combine_dual_residual(const void *y, int dtype, int S, int H, int K, int
     if (residual && !rows_ok(residual, H, b)) return MOE_ERR_INVALID_ARG;
     if (residual_no_routed_out && !rows_ok(residual_no_routed_out, H, b)) return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_combine_dual_residual");
     return to_rc(moe::launch_combine(y, dtype, S, H, K, cap, slot_of, topk_w, shared_out, residual,
                                      residual_out, residual_no_routed_out, status,
                                      static_cast<cudaStream_t>(stream)));
@@ -187,6 +208,7 @@ int moe_combine_fp8_dual_residual(const uint8_t *yq, const float *ys, int dtype,
     if (residual && !rows_ok(residual, H, b)) return MOE_ERR_INVALID_ARG;
     if (residual_no_routed_out && !rows_ok(residual_no_routed_out, H, b)) return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_combine_fp8_dual_residual");
     return to_rc(moe::launch_combine_fp8(yq, ys, dtype, S, H, K, cap, slot_of, topk_w, shared_out, residual,
                                          residual_out, residual_no_routed_out, status,
                                          static_cast<cudaStream_t>(stream)));
@@ -208,6 +230,7 @@ int moe_combine_dual_residual_backward(const void *grad_out, const void *grad_no
     if (grad_no_routed && !rows_ok(grad_no_routed, H, b)) return MOE_ERR_INVALID_ARG;
     if (grad_skip && !rows_ok(grad_skip, H, b)) return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_combine_dual_residual_backward");
     return to_rc(moe::launch_combine_backward(grad_out, grad_no_routed, y, dtype, S, H, K, cap, slot_of, topk_w,
                                               grad_y, grad_w, grad_skip, status, static_cast<cudaStream_t>(stream)));
 }
@@ -222,6 +245,7 @@ int moe_dispatch_backward(const void *grad_xd, int dtype, int S, int H, int K, i
     if ((cap > 0 && !rows_ok(grad_xd, H, b)) || !rows_ok(grad_x, H, b)) return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
     // the combine with unit weights and no epilogue: grad_x[t] = sum_k grad_xd[slot]
+    const Range range("moe_dispatch_backward");
     return to_rc(moe::launch_combine(grad_xd, dtype, S, H, K, cap, slot_of, nullptr, nullptr, nullptr, grad_x,
                                      nullptr, status, static_cast<cudaStream_t>(stream)));
 }
@@ -234,6 +258,7 @@ int moe_route_topk_backward(const int32_t *topk_idx, const float *topk_w, const 
     if (!aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4) || !aligned(grad_logits, 4))
         return MOE_ERR_INVALID_ARG;
     if ((int64_t)S * E >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    const Range range("moe_route_topk_backward");
     return to_rc(moe::launch_route_backward(topk_idx, topk_w, grad_w, S, E, K, grad_logits,
                                             static_cast<cudaStream_t>(stream), current_sms()));
 }

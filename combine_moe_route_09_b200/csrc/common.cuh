@@ -1,6 +1,7 @@
 // Shared device helpers of the sm_100a MoE routing kernels.
 #pragma once
 
+#include <atomic>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -95,6 +96,21 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
+
+// A yes/no launch setting kept per device (up to 64 devices; devices past that
+// share the last entry): starts true and is switched off for that device alone
+// when the driver refuses the launch form it guards.
+struct PerDeviceFlag {
+    static constexpr int N = 64;
+    std::atomic<int> off[N] = {};
+    static int dev_index() {
+        int d = 0;
+        if (cudaGetDevice(&d) != cudaSuccess || d < 0) d = 0;
+        return d < N ? d : N - 1;
+    }
+    bool on() const { return off[dev_index()].load(std::memory_order_relaxed) == 0; }
+    void disable() { off[dev_index()].store(1, std::memory_order_relaxed); }
+};
 
 // Launch facts per (device, kernel, block size, dynamic shared memory size):
 // how many CTAs fit on one SM.  A kernel's opt-in limit for dynamic shared

@@ -147,18 +147,9 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(const CopyArgs a) {
 // FP8 e4m3, 128-channel blocks
 // ------------------------------------------------------------------------------------------
 
-#ifndef MOE_DQ_STAGE_BUDGET
-#define MOE_DQ_STAGE_BUDGET (48 * 1024)
-#endif
-#ifndef MOE_DQ_MIN_CTAS
-#define MOE_DQ_MIN_CTAS 1
-#endif
 constexpr int DQ_MAX_STAGES = 8;
-constexpr int DQ_STAGE_BUDGET = MOE_DQ_STAGE_BUDGET;         // bytes of input ring per CTA
-#ifndef MOE_DQ_CONSUMER_WARPS
-#define MOE_DQ_CONSUMER_WARPS 4
-#endif
-constexpr int DQ_CONSUMER_WARPS = MOE_DQ_CONSUMER_WARPS;
+constexpr int DQ_STAGE_BUDGET = 48 * 1024;                   // bytes of input ring per CTA
+constexpr int DQ_CONSUMER_WARPS = 4;
 constexpr int DQ_CONSUMERS = DQ_CONSUMER_WARPS * 32;
 constexpr int DQ_THREADS = DQ_CONSUMERS + 32;
 constexpr int DQ_UNIT = 16;                                  // channels of one thread unit
@@ -166,13 +157,7 @@ constexpr int DQ_UNITS = 2;                                  // units per thread
 constexpr int DQ_SPAN = DQ_CONSUMERS * DQ_UNIT;              // channels between a thread's units
 constexpr int DQ_MAX_BLOCKS = DQ_UNITS * DQ_SPAN / 128;      // 128-channel blocks per item
 constexpr int DQ_HDR = 128;                                  // per-stage header: the token's K slots
-#ifndef MOE_DQ_BULK
-#define MOE_DQ_BULK 1
-#endif
-#ifndef MOE_DQ_OUT_BUFS
-#define MOE_DQ_OUT_BUFS 2
-#endif
-constexpr int DQ_OUT_BUFS = MOE_DQ_OUT_BUFS;                 // bulk-store path: output staging buffers
+constexpr int DQ_OUT_BUFS = 2;                 // bulk-store path: output staging buffers
 constexpr int DQ_BULK_MIN_ITEMS_PER_SM = 16;                 // bulk-store path from this many items per SM
 
 struct Fp8Args {
@@ -258,7 +243,7 @@ __device__ __forceinline__ U4 quant16(const float (&f)[16], float s) {
 // leave through TMA bulk stores from a shared-memory staging buffer (one
 // elected thread issues them) instead of per-thread 16-byte stores.
 template <bool IN_F32, int KT, bool BULK>
-__global__ void __launch_bounds__(DQ_THREADS, MOE_DQ_MIN_CTAS) dispatch_fp8_kernel(const Fp8Args a) {
+__global__ void __launch_bounds__(DQ_THREADS) dispatch_fp8_kernel(const Fp8Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     // layout: [stages][header (K slots) | bpc*128*esz input bytes]
     //         | BULK: [DQ_OUT_BUFS][bpc*128 codes | bpc*4 scales, padded to 16] | barriers
@@ -531,7 +516,7 @@ cudaError_t launch_dispatch(const void *x, int dtype, int S, int H, int K, const
     cudaError_t ae = cudaGetDevice(&dev);
     if (ae == cudaSuccess) ae = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
     if (ae != cudaSuccess) return ae;
-    const bool bulk = MOE_DQ_BULK != 0 && nitems >= (long long)DQ_BULK_MIN_ITEMS_PER_SM * sm_count;
+    const bool bulk = nitems >= (long long)DQ_BULK_MIN_ITEMS_PER_SM * sm_count;
     const size_t smem = (size_t)a.stages * a.stage + (bulk ? (size_t)DQ_OUT_BUFS * a.obuf : 0) + 2 * DQ_MAX_STAGES * 8;
     auto go = [&](auto kern) -> cudaError_t {
         static KernelSlots<decltype(kern)> slots;

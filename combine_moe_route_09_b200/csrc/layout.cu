@@ -522,23 +522,14 @@ __global__ void __launch_bounds__(LT_THREADS)
 // tiles below it.  No global scratch, no atomics, no spin-wait.
 // ------------------------------------------------------------------------------------------
 
-#ifndef MOE_LC_WARPS
-#define MOE_LC_WARPS 16
-#endif
-#ifndef MOE_LC_MAX_CTAS
-#define MOE_LC_MAX_CTAS 16
-#endif
-constexpr int LC_WARPS = MOE_LC_WARPS;
+constexpr int LC_WARPS = 16;
 constexpr int LC_THREADS = LC_WARPS * 32;
-#ifndef MOE_LC_ITEMS
-#define MOE_LC_ITEMS 4
-#endif
-constexpr int LC_ITEMS = MOE_LC_ITEMS;
+constexpr int LC_ITEMS = 4;
 constexpr int LC_TILE = LC_THREADS * LC_ITEMS;  // 2048 pairs per CTA
 // 16 CTAs: above the portable cluster size of 8, allowed per function (the
 // layout falls back to the other paths where the device refuses it).  In the
 // DeepSeek-V3-shaped prefill step, 16 CTAs of 512 threads beat 8 CTAs of 1024.
-constexpr int LC_MAX_CTAS = MOE_LC_MAX_CTAS;
+constexpr int LC_MAX_CTAS = 16;
 
 __global__ void __launch_bounds__(LC_THREADS)
     layout_cluster_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P, int64_t cap,
@@ -765,8 +756,8 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     cudaError_t e = slots.prepare(&layout_cluster_kernel, LC_THREADS, smem, &sms, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaSuccess;
-    static int pdl_ok = 1, cluster_ok = 1;
-    if (!cluster_ok) return cudaSuccess;
+    static PerDeviceFlag pdl_ok, cluster_ok;
+    if (!cluster_ok.on()) return cudaSuccess;
     if (dry) {
         *launched = true;
         return cudaSuccess;
@@ -775,7 +766,7 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
         e = cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
-            cluster_ok = 0;
+            cluster_ok.disable();
             return cudaSuccess;
         }
     }
@@ -792,19 +783,19 @@ static cudaError_t launch_layout_cluster(const int32_t *topk_idx, int npairs, in
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_ok ? 2 : 1;
+    cfg.numAttrs = pdl_ok.on() ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, topk_idx, npairs, E, R, P, cap, counts, offsets,
                            rank_offsets, slot_of, row_src, status);
-    if (e != cudaSuccess && pdl_ok) {
-        (void)cudaGetLastError();  // the pair was refused: launch without PDL from now on
-        pdl_ok = 0;
+    if (e != cudaSuccess && cfg.numAttrs == 2) {
+        (void)cudaGetLastError();  // the pair was refused: launch without PDL on this device from now on
+        pdl_ok.disable();
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, topk_idx, npairs, E, R, P, cap, counts, offsets,
                                rank_offsets, slot_of, row_src, status);
     }
     if (e != cudaSuccess) {
-        (void)cudaGetLastError();  // no cluster launch here: the other paths from now on
-        cluster_ok = 0;
+        (void)cudaGetLastError();  // no cluster launch on this device: the other paths from now on
+        cluster_ok.disable();
         return cudaSuccess;
     }
     *launched = true;
@@ -830,7 +821,7 @@ static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int 
     }
     // Cooperative (all CTAs co-resident, for the grid barrier) and, where the
     // driver accepts the pair, programmatic serialisation too (see pdl_wait).
-    static int pdl_ok = 1;
+    static PerDeviceFlag pdl_ok;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(LT_THREADS);
@@ -842,12 +833,12 @@ static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int 
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_ok ? 2 : 1;
+    cfg.numAttrs = pdl_ok.on() ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts,
                            offsets, rank_offsets, slot_of, row_src, status);
-    if (e != cudaSuccess && pdl_ok) {
-        (void)cudaGetLastError();  // the pair was refused: launch cooperative only from now on
-        pdl_ok = 0;
+    if (e != cudaSuccess && cfg.numAttrs == 2) {
+        (void)cudaGetLastError();  // the pair was refused: launch cooperative only on this device from now on
+        pdl_ok.disable();
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts,
                                offsets, rank_offsets, slot_of, row_src, status);
@@ -859,12 +850,10 @@ static cudaError_t launch_layout_fused(const int32_t *topk_idx, int npairs, int 
 int layout_kernel_count(int S, int E, int K) {
     const int npairs = S * K;
     bool one = false;
-#ifndef MOE_NO_CLUSTER_LAYOUT
     if (launch_layout_cluster(nullptr, npairs, E, 1, 0, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                               nullptr, &one, true) != cudaSuccess)
         return -1;
     if (one) return 1;
-#endif
     if (launch_layout_fused(nullptr, npairs, E, 1, 0, 0, layout_tiles(npairs), nullptr, nullptr, nullptr, nullptr,
                             nullptr, nullptr, nullptr, nullptr, nullptr, &one, true) != cudaSuccess)
         return -1;
@@ -880,12 +869,10 @@ cudaError_t launch_layout(const int32_t *topk_idx, int S, int E, int K, int R, i
     auto *hdr = reinterpret_cast<LayoutHeader *>(workspace);
     auto *hist = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(workspace) + LT_HEADER);
     bool launched = false;
-#ifndef MOE_NO_CLUSTER_LAYOUT
     cudaError_t ce = launch_layout_cluster(topk_idx, npairs, E, R, P, cap, counts, offsets, rank_offsets, slot_of,
                                            row_src, status, st, &launched);
     if (ce != cudaSuccess) return ce;
     if (launched) return cudaSuccess;
-#endif
     cudaError_t fe = launch_layout_fused(topk_idx, npairs, E, R, P, cap, T, hist, hdr, counts, offsets,
                                          rank_offsets, slot_of, row_src, status, st, &launched);
     if (fe != cudaSuccess) return fe;

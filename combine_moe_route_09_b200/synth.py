@@ -42,7 +42,7 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_ZIPF_FILE = os.path.join(os.path.dirname(_HERE), "tests", "golden", "zipf_alpha.json")
+_ZIPF_FILE = os.path.join(_HERE, "zipf_alpha.json")
 
 
 @dataclass(frozen=True)

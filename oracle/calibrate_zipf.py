@@ -5,7 +5,7 @@ alpha * (-1.1 * ln r_e) to every token's logits, r_e a seeded permutation of
 1..E, and wants the busiest expert to receive about 4x the mean load.  This
 script routes the seeded logits with the oracle for each trial alpha, bisects
 on max/mean of the oracle's per-expert counts, and writes the result to
-tests/golden/zipf_alpha.json, which the input generator reads.
+combine_moe_route_09_b200/zipf_alpha.json, which the input generator reads.
 
 Run:  python -m oracle.calibrate_zipf
 """
@@ -23,7 +23,7 @@ import oracle  # noqa: E402
 from combine_moe_route_09_b200 import synth  # noqa: E402
 
 OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                   "tests", "golden", "zipf_alpha.json")
+                   "combine_moe_route_09_b200", "zipf_alpha.json")
 
 
 def load_ratio(w: synth.Workload, alpha: float) -> float:

@@ -64,6 +64,35 @@ def _run_bench(env_extra, *args):
                           text=True, env=env, timeout=600, cwd=ROOT)
 
 
+def bench_threads() -> int:
+    sys.path.insert(0, ROOT)
+    import bench
+
+    return bench.host_threads()
+
+
+def test_threaded_oracle_pass_equals_single_threaded():
+    """The CPU baseline splits the per-token steps over threads by token range;
+    the result must be the single-threaded pass, bit for bit."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_moe_route_09_b200 import synth
+
+    for key in ("1", "2b"):
+        w = synth.WORKLOADS[key]
+        inp = bench.host_inputs(w)
+        a = bench.oracle_pass(w, inp, w.S, 1)
+        b = bench.oracle_pass(w, inp, w.S, 3)
+        for k in ("topk_idx", "topk_w", "xd", "out"):
+            assert np.array_equal(a[k], b[k]), (key, k)
+        for k in ("slot_of", "row_src", "counts", "offsets"):
+            assert np.array_equal(a["layout"][k], b["layout"][k]), (key, k)
+        if a["out_no_routed"] is not None:
+            assert np.array_equal(a["out_no_routed"], b["out_no_routed"])
+
+
 def test_reference_arm_line_contract():
     r = _run_bench({}, "--impl", "reference", "--workload", "1", "--steps", "3", "--warmup", "3")
     assert r.returncode == 0, r.stderr
@@ -72,7 +101,7 @@ def test_reference_arm_line_contract():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["steps"] == 3 and d["warmup"] == 3
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == bench_threads()
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "tiny_fp32"
