@@ -458,7 +458,8 @@ def measure_workload(w, args, world, local_rank, device, windows, e2e: bool):
     pinned = {k: synth.to_torch(v).pin_memory() for k, v in inp.items()}
     d = {k: v.to(device, non_blocking=True) for k, v in pinned.items()}
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
-    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device)
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", device=device,
+                    fused=args.fused)
     sh, rs = (d["shared"], d["residual"]) if w.fused else (None, None)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -466,19 +467,24 @@ def measure_workload(w, args, world, local_rank, device, windows, e2e: bool):
     torch.cuda.synchronize()
     if buf.read_status() != 0:
         raise RuntimeError("device status flagged a problem during warm-up")
-    graph = None
+    K = args.steps
+    graph, gsteps = None, 1
     if args.graph:
-        graph = buf.capture(d["logits"], d["x"], d["y"], sh, rs)
+        # consecutive steps captured in one graph, as a model's layers would be;
+        # each kernel still waits for the one before it
+        gsteps = max(1, min(args.graph_steps, K))
+        while K % gsteps:
+            gsteps -= 1
+        graph = buf.capture(d["logits"], d["x"], d["y"], sh, rs, steps=gsteps)
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
         if buf.read_status() != 0:
-            raise RuntimeError("device status flagged a problem in the captured step")
+            raise RuntimeError("device status flagged a problem in the captured steps")
     step = graph.replay if graph is not None else (lambda: buf.step(d["logits"], d["x"], d["y"], sh, rs))
 
-    K = args.steps
     h0 = time.perf_counter()
-    win_ms = time_windows(step, K, windows, world, device)
+    win_ms = time_windows(step, K // gsteps, windows, world, device)
     host_us = (time.perf_counter() - h0) / (K * windows) * 1e6
     phases = buf.step_phases(d["logits"], d["x"], d["y"], sh, rs)
     Kp = max(1, min(K, 50))
@@ -553,8 +559,10 @@ def measure_workload(w, args, world, local_rank, device, windows, e2e: bool):
         "phases_marginal": _phase_table(marginal, ab, peak),
         "phases_eager": _phase_table({k: statistics.median(v) for k, v in eager.items()}, ab, peak),
         "gpu_launches_per_step": buf.kernels_per_step,
-        "host_enqueue_us_per_step": host_us,
-        "graph": graph is not None,
+        "host_enqueue_us_per_step": host_us * gsteps,
+        "graph": graph is not None, "graph_steps": gsteps,
+        "plan": "fused route+layout+dispatch kernel" if buf.fused else "separate route, layout, dispatch kernels",
+        "plan_timings_us": buf.plan_timings_us,
     }
     res["_buf"], res["_inp"], res["_e2e"], res["_peak"] = buf, inp, e2e_res, (peak, peak_kind)
     return res
@@ -615,12 +623,14 @@ def run_ours(args, w, rank, world, local_rank):
         "roofline": roofline, "e2e": e2e,
         "gpu_launches": K * head["gpu_launches_per_step"], "clocks": clocks,
         "timing": ("value: median over windows of exactly K steps (barrier + synchronize around each window), "
-                   + ("each step one CUDA-graph replay" if head["graph"] else "eager calls")
+                   + (f"{head['graph_steps']} consecutive steps per CUDA-graph replay" if head["graph"]
+                      else "eager calls")
                    + "; phases: CUDA event nodes between the kernels inside a graph of min(K, 50) steps; "
                      "phases_marginal: leave-one-out graphs (a graph of the first j+1 phases minus one of the "
                      "first j), consecutive kernels overlapping as in the step; phases_eager: eager calls with "
                      "an event between kernels"),
         "host_enqueue_us_per_step": head["host_enqueue_us_per_step"],
+        "plan": head["plan"], "plan_timings_us": head["plan_timings_us"],
         "workloads": others,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -892,6 +902,11 @@ def main(argv=None):
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time the value pass as CUDA-graph replays of one step (default; "
                          "--no-graph times eager calls)")
+    ap.add_argument("--graph-steps", type=int, default=10,
+                    help="consecutive steps captured in one CUDA graph (a divisor of --steps is used)")
+    ap.add_argument("--fused", action=argparse.BooleanOptionalAction, default=None,
+                    help="route + layout + dispatch as one kernel where it applies (--fused), never "
+                         "(--no-fused), or (default) whichever of the two plans MoeBuffer times faster")
     ap.add_argument("--mode", default="forward", choices=["forward", "backward", "fp8_combine", "router"],
                     help="forward: the routing pass (default); backward: its training backward; "
                          "fp8_combine: the combine over FP8 expert outputs; router: both routers")

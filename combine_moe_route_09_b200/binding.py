@@ -42,6 +42,10 @@ SIGNATURES = {
     "moe_combine_dual_residual_backward": (_I, [_P, _P, _P, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_backward": (_I, [_P, _I, _I, _I, _I, _L, _P, _P, _P, _P]),
     "moe_route_topk_backward": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_route_dispatch_workspace": (_Z, [_I, _I, _I]),
+    "moe_route_dispatch_kernels": (_I, [_I, _I, _I, _I, _I, _I]),
+    "moe_route_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _L,
+                                _P, _Z, _P, _P]),
     "moe_error_string": (ctypes.c_char_p, [_I]),
     "moe_capacity": (_L, [_I, _I, _I, _I]),
 }
@@ -95,6 +99,14 @@ def _dev(t: torch.Tensor, name: str, dtypes, shape=None):
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
     return t
+
+
+def _dtype_code_of(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return MOE_DTYPE_F32
+    if dt == torch.bfloat16:
+        return MOE_DTYPE_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {dt}")
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -244,6 +256,70 @@ def moe_dispatch_layout_static(topk_idx: torch.Tensor, E: int, R: int, token_pad
         _ptr(out.rank_offsets), _ptr(out.slot_of), _ptr(out.row_src), cap, _ptr(status),
         _stream(stream, dev)))
     return out._replace(cap=cap)
+
+
+def moe_route_dispatch_workspace(S: int, E: int, K: int) -> int:
+    return int(lib().moe_route_dispatch_workspace(S, E, K))
+
+
+def moe_route_dispatch_kernels(S: int, H: int, E: int, K: int, dtype: torch.dtype = torch.bfloat16,
+                               quant: int = MOE_QUANT_NONE) -> int:
+    """1 when moe_route_dispatch runs as one fused kernel for these sizes on the
+    current device, else the number of separate kernels (3 or 4)."""
+    return int(lib().moe_route_dispatch_kernels(S, H, E, K, _dtype_code_of(dtype), quant))
+
+
+def moe_route_dispatch(logits: torch.Tensor, x: torch.Tensor, K: int, R: int, token_padding: int = 0,
+                       quant: int = MOE_QUANT_NONE, cap: Optional[int] = None, *, topk_idx=None, topk_w=None,
+                       layout: Optional[Layout] = None, xd=None, xs=None, workspace=None, status=None,
+                       stream=None):
+    """Router top-K, dispatch layout and dispatch in one call (one kernel when the
+    batch fits).  Returns (topk_idx, topk_w, layout, xd, xs), exactly what
+    moe_route_topk, moe_dispatch_layout and moe_dispatch would return.
+
+    ``workspace`` (uint8, >= moe_route_dispatch_workspace bytes) must be
+    zero-filled before its first use; a fresh one is allocated if not given."""
+    _dev(logits, "logits", (torch.float32,))
+    _dev(x, "x", _ACT)
+    S, E = logits.shape
+    H = x.shape[1]
+    _dev(x, "x", _ACT, (S, H))
+    dev = x.device
+    if cap is None:
+        cap = moe_capacity(S, E, K, token_padding)
+    i32 = dict(dtype=torch.int32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty((S, K), **i32)
+    if topk_w is None:
+        topk_w = torch.empty((S, K), dtype=torch.float32, device=dev)
+    _dev(topk_idx, "topk_idx", (torch.int32,), (S, K))
+    _dev(topk_w, "topk_w", (torch.float32,), (S, K))
+    if layout is None:
+        layout = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                        torch.empty((S, K), **i32), torch.empty(max(cap, 0), **i32), cap)
+    if quant == MOE_QUANT_FP8_E4M3_B128:
+        if xd is None:
+            xd = torch.empty((cap, H), dtype=torch.float8_e4m3fn, device=dev)
+        if xs is None:
+            xs = torch.empty((cap, H // 128), dtype=torch.float32, device=dev)
+        _dev(xd, "xd", (torch.float8_e4m3fn, torch.uint8), (cap, H))
+        _dev(xs, "xs", (torch.float32,), (cap, H // 128))
+    else:
+        if xd is None:
+            xd = torch.empty((cap, H), dtype=x.dtype, device=dev)
+        _dev(xd, "xd", (x.dtype,), (cap, H))
+    need = moe_route_dispatch_workspace(S, E, K)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", (torch.uint8,))
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    _check("moe_route_dispatch", lib().moe_route_dispatch(
+        _ptr(logits), _ptr(x), _dtype_code(x), S, H, E, K, R, token_padding, quant, _ptr(topk_idx), _ptr(topk_w),
+        _ptr(layout.counts), _ptr(layout.offsets), _ptr(layout.rank_offsets), _ptr(layout.slot_of),
+        _ptr(layout.row_src), _ptr(xd), _ptr(xs), cap, _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream, dev)))
+    return topk_idx, topk_w, layout._replace(cap=cap), xd, xs
 
 
 def moe_dispatch(x: torch.Tensor, slot_of: torch.Tensor, cap: int, quant: int = MOE_QUANT_NONE,

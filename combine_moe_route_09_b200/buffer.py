@@ -32,7 +32,8 @@ class MoeBuffer:
     """
 
     def __init__(self, S: int, H: int, K: int, E: int, R: int = 1, token_padding: int = 0,
-                 dtype: torch.dtype = torch.bfloat16, fp8: bool = False, device="cuda"):
+                 dtype: torch.dtype = torch.bfloat16, fp8: bool = False, device="cuda",
+                 fused: Optional[bool] = None):
         if dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("activations must be float32 or bfloat16")
         self.S, self.H, self.K, self.E, self.R, self.P = S, H, K, E, R, token_padding
@@ -50,7 +51,7 @@ class MoeBuffer:
         self.layout = B.Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32),
                                torch.empty(R + 1, **i32), torch.empty((S, K), **i32),
                                torch.empty(self.cap, **i32), self.cap)
-        ws = B.moe_dispatch_layout_workspace(S, E, K)
+        ws = max(B.moe_dispatch_layout_workspace(S, E, K), B.moe_route_dispatch_workspace(S, E, K))
         self.workspace = torch.zeros(max(ws, 256), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
         if fp8:
@@ -73,10 +74,25 @@ class MoeBuffer:
         self._p_slot, self._p_xd = p(L.slot_of), p(self.xd)
         self._p_xs = p(self.xs) if fp8 else None
         self._p_out, self._p_rnr = p(self.out), p(self.out_no_routed)
+        self._rd_args = (S, H, E, K, R, token_padding, self.quant, p(self.topk_idx), p(self.topk_w), p(L.counts),
+                         p(L.offsets), p(L.rank_offsets), p(L.slot_of), p(L.row_src), self._p_xd, self._p_xs,
+                         self.cap, p(self.workspace), self.workspace.numel(), p(self.status))
+        # route + layout + dispatch as one fused kernel when it applies to these sizes
+        # on this device: fused=True forces it, False never uses it, None (default)
+        # times both plans once (they give identical outputs) and keeps the faster
+        with torch.cuda.device(self.device):
+            applies = B.moe_route_dispatch_kernels(S, H, E, K, dtype, self.quant) == 1
+        self.fused = applies and fused is not False
+        self.plan_timings_us = None
+        if applies and fused is None:
+            self._choose_plan()
 
     @property
     def kernels_per_step(self) -> int:
-        """Kernels one step launches: route 1, layout 1 or 2, dispatch 1, combine 1."""
+        """Kernels one step launches: fused route + layout + dispatch 1, combine 1; or
+        route 1, layout 1 or 2, dispatch 1, combine 1."""
+        if self.fused:
+            return 2
         with torch.cuda.device(self.device):
             return 3 + B.moe_dispatch_layout_kernels(self.S, self.E, self.K)
 
@@ -114,6 +130,15 @@ class MoeBuffer:
         B._check("moe_dispatch_layout", self._lib.moe_dispatch_layout(*args, self._stream(stream)))
         return self.layout
 
+    def route_dispatch(self, logits: torch.Tensor, x: torch.Tensor, stream=None):
+        """route + plan + dispatch as one call (one kernel when the batch fits)."""
+        pl = self._in(logits, "logits", (torch.float32,), (self.S, self.E))
+        px = self._in(x, "x", (self.dtype,), (self.S, self.H))
+        a = self._rd_args
+        B._check("moe_route_dispatch", self._lib.moe_route_dispatch(
+            pl, px, self._dt, *a, self._stream(stream)))
+        return self.xd, self.xs
+
     def dispatch(self, x: torch.Tensor, stream=None):
         px = self._in(x, "x", (self.dtype,), (self.S, self.H))
         B._check("moe_dispatch", self._lib.moe_dispatch(px, self._dt, self.S, self.H, self.K, self._p_slot,
@@ -135,6 +160,11 @@ class MoeBuffer:
     def step_phases(self, logits, x, y, shared_out=None, residual=None, stream=None):
         """The calls of one full pass, in order, as (phase name, zero-argument call)
         pairs; running them in order is one step (y = expert outputs)."""
+        if self.fused:
+            return [
+                ("route_dispatch", lambda: self.route_dispatch(logits, x, stream)),
+                ("combine", lambda: self.combine(y, shared_out, residual, stream=stream)),
+            ]
         return [
             ("route", lambda: self.route(logits, stream)),
             ("layout", lambda: self.plan(stream=stream)),
@@ -148,21 +178,63 @@ class MoeBuffer:
             call()
         return self.out, (self.out_no_routed if (shared_out is not None and residual is not None) else None)
 
-    def capture(self, logits, x, y, shared_out=None, residual=None):
-        """Records one step into a CUDA graph and returns it (``graph.replay()``
-        reruns the step).  The graph reads the given input tensors and writes this
-        buffer's outputs at fixed addresses: refill the inputs in place between
-        replays.  Run one eager step first (kernel attributes are set on first use)."""
+    def capture(self, logits, x, y, shared_out=None, residual=None, steps: int = 1):
+        """Records `steps` consecutive steps into a CUDA graph and returns it
+        (``graph.replay()`` reruns them).  The graph reads the given input tensors
+        and writes this buffer's outputs at fixed addresses: refill the inputs in
+        place between replays.  Run one eager step first (kernel attributes are set
+        on first use)."""
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self.step(logits, x, y, shared_out, residual)
+            for _ in range(steps):
+                self.step(logits, x, y, shared_out, residual)
         return g
+
+    def _choose_plan(self, calls: int = 10, reps: int = 5):
+        """Times route + layout + dispatch both ways -- the fused kernel and the
+        separate kernels -- on synthetic inputs of this buffer's shapes, each as a
+        CUDA graph of `calls` back-to-back calls, and keeps the faster (median of
+        `reps`).  Both plans write identical outputs; only the speed differs."""
+        dev = self.device
+        gen = torch.Generator(device=dev).manual_seed(0)
+        logits = torch.randn((self.S, self.E), generator=gen, device=dev)
+        x = torch.randn((self.S, self.H), generator=gen, device=dev).to(self.dtype)
+        side = torch.cuda.Stream(dev)
+        times = {}
+        with torch.cuda.device(dev):
+            for fused in (True, False):
+                self.fused = fused
+                run = (lambda: self.route_dispatch(logits, x)) if fused else \
+                    (lambda: (self.route(logits), self.plan(), self.dispatch(x)))
+                run()
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                side.wait_stream(torch.cuda.current_stream(dev))
+                with torch.cuda.graph(g, stream=side):
+                    for _ in range(calls):
+                        run()
+                g.replay()
+                torch.cuda.synchronize(dev)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ts = []
+                for _ in range(reps):
+                    a.record()
+                    g.replay()
+                    b.record()
+                    torch.cuda.synchronize(dev)
+                    ts.append(a.elapsed_time(b) * 1e3 / calls)
+                del g
+                times["fused" if fused else "separate"] = sorted(ts)[len(ts) // 2]
+        self.fused = times["fused"] <= times["separate"]
+        self.plan_timings_us = times
+        self._seen.clear()
+        self.read_status()
 
     def read_status(self) -> int:
         """Reads and clears the device status word (synchronises).  After a
-        timeout the layout workspace header is zeroed again, as its contract asks."""
+        timeout the workspace is zeroed again, as its contract asks."""
         v = int(self.status.item())
         self.status.zero_()
         if v & B.MOE_STATUS_TIMEOUT:
-            self.workspace[:256].zero_()
+            self.workspace.zero_()
         return v

@@ -147,6 +147,53 @@ int moe_dispatch_layout(const int32_t *topk_idx, int S, int E, int K, int R, int
                                     static_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_route_dispatch_workspace(int S, int E, int K) {
+    if (S < 0 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > MOE_MAX_TOPK) return 0;
+    if ((int64_t)S * K >= ((int64_t)1 << 31)) return 0;
+    return moe::route_dispatch_workspace_bytes(S, E, K);
+}
+
+int moe_route_dispatch_kernels(int S, int H, int E, int K, int dtype, int quant) {
+    if (S < 1 || H < 1 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > E || K > MOE_MAX_TOPK || esize(dtype) == 0 ||
+        (quant != MOE_QUANT_NONE && quant != MOE_QUANT_FP8_E4M3_B128) || (int64_t)S * K >= ((int64_t)1 << 31))
+        return 0;
+    return moe::route_dispatch_kernel_count(S, H, E, K, dtype, quant);
+}
+
+int moe_route_dispatch(const float *logits, const void *x, int dtype, int S, int H, int E, int K, int R,
+                       int token_padding, int quant, int32_t *topk_idx, float *topk_w, int32_t *counts,
+                       int32_t *offsets, int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src, void *xd,
+                       float *xs, int64_t cap, void *workspace, size_t workspace_bytes, int32_t *status,
+                       void *stream) {
+    // the checks of moe_route_topk, moe_dispatch_layout and moe_dispatch together
+    const int b = esize(dtype);
+    if (S < 0 || H < 1 || E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > E || K > MOE_MAX_TOPK || R < 1 ||
+        E % R != 0 || token_padding < 0 || b == 0 || cap < 0 || cap >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (quant != MOE_QUANT_NONE && quant != MOE_QUANT_FP8_E4M3_B128) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * K + (int64_t)E * (token_padding > 0 ? token_padding - 1 : 0) >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)S * E >= ((int64_t)1 << 40) || (int64_t)S * H >= ((int64_t)1 << 40)) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !rank_offsets || !workspace) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!logits || !topk_idx || !topk_w || !slot_of || !rows_ok(x, H, b))) return MOE_ERR_INVALID_ARG;
+    if (cap > 0 && !row_src) return MOE_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || workspace_bytes < moe::route_dispatch_workspace_bytes(S, E, K))
+        return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {logits, topk_idx, topk_w, counts, offsets, rank_offsets, slot_of, row_src, status};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+    if (quant == MOE_QUANT_NONE) {
+        if (xs || (cap > 0 && S > 0 && !rows_ok(xd, H, b))) return MOE_ERR_INVALID_ARG;
+    } else {
+        if (H % 128 != 0 || (cap > 0 && S > 0 && (!rows_ok(xd, H, 1) || !xs || !aligned(xs, 4))))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const Range range("moe_route_dispatch");
+    return to_rc(moe::launch_route_dispatch(logits, x, dtype, S, H, E, K, R, token_padding, quant, topk_idx, topk_w,
+                                            counts, offsets, rank_offsets, slot_of, row_src, xd, xs, cap, workspace,
+                                            status, static_cast<cudaStream_t>(stream), current_sms()));
+}
+
 int moe_dispatch(const void *x, int dtype, int S, int H, int K, const int32_t *slot_of, int quant,
                  void *xd, float *xs, int64_t cap, int32_t *status, void *stream) {
     const int b = esize(dtype);

@@ -25,6 +25,18 @@ inline size_t layout_workspace_bytes(int S, int E, int K) {
     return LT_HEADER + ((hist + 255) / 256) * 256;
 }
 
+// Fused route + layout + dispatch: scratch header, then [RD_MAX_CTAS][E rounded up to 4] int32.
+constexpr size_t RD_HEADER_BYTES = LT_HEADER;
+constexpr int RD_MAX_CTAS = 512;
+size_t route_dispatch_workspace_bytes(int S, int E, int K);
+// Kernels moe_route_dispatch launches for these sizes on the current device (1 fused, else 3 or 4; -1: CUDA error).
+int route_dispatch_kernel_count(int S, int H, int E, int K, int dtype, int quant);
+cudaError_t launch_route_dispatch(const float *logits, const void *x, int dtype, int S, int H, int E, int K, int R,
+                                  int P, int quant, int32_t *topk_idx, float *topk_w, int32_t *counts,
+                                  int32_t *offsets, int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src,
+                                  void *xd, float *xs, int64_t cap, void *workspace, int32_t *status,
+                                  cudaStream_t st, int sms);
+
 cudaError_t launch_route_topk(const float *logits, int S, int E, int K, int32_t *idx, float *w,
                               cudaStream_t st, int sms);
 

@@ -31,35 +31,11 @@
 // (ascending t*K + k) with the same expert: a stable counting sort.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "layout_core.cuh"
 #include "tma.cuh"
 
 namespace moe {
 
-struct LayoutHeader {
-    unsigned int ticket;   // two-kernel path: arrival ticket, reset by the last CTA
-    unsigned int count;    // fused path: grid-barrier arrivals, reset by the last arriver
-    unsigned int gen;      // fused path: grid-barrier generation (only ever incremented)
-};
-
-__device__ __forceinline__ int pad_count(int c, int P) { return P > 0 ? ((c + P - 1) / P) * P : c; }
-
-// Lanes of the warp holding the same expert id as this lane (e = -1: none).
-// One ballot per bit of the id (ids below 2^nbits) plus one for validity: a
-// fixed, short sequence, where __match_any_sync takes longer the more
-// distinct values the warp holds.
-__device__ __forceinline__ unsigned expert_peers(int e, int nbits) {
-    unsigned peers = __ballot_sync(FULL, e >= 0);
-    if (e < 0) peers = ~peers;
-    for (int b = 0; b < nbits; ++b) {
-        const bool bit = (e >> b) & 1;
-        const unsigned m = __ballot_sync(FULL, bit);
-        peers &= bit ? m : ~m;
-    }
-    return peers;
-}
-
-// Bits that cover every expert id below E.
-__device__ __forceinline__ int expert_bits(int E) { return E > 1 ? 32 - __clz(E - 1) : 0; }
 
 __global__ void __launch_bounds__(LT_THREADS)
     layout_hist_kernel(const int32_t *__restrict__ topk_idx, int npairs, int E, int R, int P,
@@ -291,27 +267,11 @@ __global__ void __launch_bounds__(LT_THREADS)
 
 constexpr int LF_MAX_HIST = 64 * 1024;  // T * E entries a CTA may scan in phase 2
 
-// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  Sense
-// reversal: read the generation, arrive; the last arriver resets the count and
-// bumps the generation; the others wait (bounded) for the bump.  False on timeout.
+// Grid-wide barrier of the whole CTA (see grid_arrive_wait).
 __device__ bool grid_barrier(LayoutHeader *hdr, int32_t *status) {
     __shared__ int s_ok;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        const unsigned gen = *(volatile unsigned *)&hdr->gen;
-        __threadfence();
-        const unsigned prev = atomicAdd(&hdr->count, 1u);
-        if (prev == gridDim.x - 1) {
-            *(volatile unsigned *)&hdr->count = 0u;
-            __threadfence();
-            atomicExch(&hdr->gen, gen + 1u);
-        } else {
-            ok = wait_changed_for(&hdr->gen, gen, status, MOE_WAIT_NS) ? 1 : 0;
-        }
-        __threadfence();
-        s_ok = ok;
-    }
+    if (threadIdx.x == 0) s_ok = grid_arrive_wait(hdr, status) ? 1 : 0;
     __syncthreads();
     return s_ok != 0;
 }

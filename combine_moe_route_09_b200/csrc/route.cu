@@ -1,31 +1,14 @@
-// Router top-K gating: one warp per logits row.
+// Router top-K gating: one warp per logits row (the per-row routine is in
+// route_core.cuh, shared with the fused route + dispatch kernel).
 //
 // "Efficient and portable mixture-of-experts communication", Introduction:
 // each token is sent to the K experts with the highest router scores, and the
 // expert outputs are added with weights from the router's distribution.
-//
-// Each lane holds ceil(E/32) logits of the row (expert e = lane + 32*j) in
-// registers as ordered 32-bit keys: ordered() maps fp32 to uint32
-// monotonically (after -0.0 -> +0.0), so a larger key is a larger logit.
-// Round k of K: the warp max of the keys (redux.sync.max), then the lowest
-// expert id holding that key (redux.sync.min over each lane's lowest
-// candidate) -- ties go to the lower id -- and that key is cleared to 0,
-// below every real key.  The softmax over the K selected logits runs on lanes
-// 0..K-1.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "route_core.cuh"
 
 namespace moe {
-
-__device__ __forceinline__ uint32_t ordered_bits(float v) {
-    uint32_t u = __float_as_uint(v);
-    if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float from_ordered(uint32_t o) {
-    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
-}
 
 template <int NPER>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int S,
@@ -36,39 +19,14 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < S; t += warps) {
-        const float *row = logits + (size_t)t * E;
         uint32_t key[NPER];
-#pragma unroll
-        for (int j = 0; j < NPER; ++j) {
-            const int e = lane + 32 * j;
-            key[j] = e < E ? ordered_bits(__ldg(row + e)) : 0u;
-        }
-        uint32_t my_key = 0, top = 0;
-        int my_e = 0;
-        for (int k = 0; k < K; ++k) {
-            uint32_t m = key[0];
-#pragma unroll
-            for (int j = 1; j < NPER; ++j) m = max(m, key[j]);
-            const uint32_t best = __reduce_max_sync(FULL, m);
-            uint32_t cand = 0xffffffffu;
-#pragma unroll
-            for (int j = NPER - 1; j >= 0; --j) cand = key[j] == best ? (uint32_t)(lane + 32 * j) : cand;
-            const uint32_t win = __reduce_min_sync(FULL, cand);
-            if (k == 0) top = best;
-            if (lane == k) {
-                my_key = best;
-                my_e = (int)win;
-            }
-#pragma unroll
-            for (int j = 0; j < NPER; ++j) key[j] = (uint32_t)(lane + 32 * j) == win ? 0u : key[j];
-        }
-        const float ex = lane < K ? expf(from_ordered(my_key) - from_ordered(top)) : 0.f;
-        float sum = ex;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+        load_route_keys<NPER>(logits + (size_t)t * E, E, lane, key);
+        int my_e;
+        float my_w;
+        topk_softmax<NPER>(key, K, lane, my_e, my_w);
         if (lane < K) {
             topk_idx[(size_t)t * K + lane] = my_e;
-            topk_w[(size_t)t * K + lane] = __fdiv_rn(ex, sum);
+            topk_w[(size_t)t * K + lane] = my_w;
         }
     }
 }

@@ -138,6 +138,12 @@ __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrives at named barrier `id` without waiting (the other side waits with
+// named_bar over the same `count`).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Named barrier that also ANDs a predicate over its `count` threads, so that a
 // decision to leave a loop is taken by all of them together.
 __device__ __forceinline__ bool named_bar_and(int id, int count, bool p) {

@@ -12,7 +12,8 @@
  *   moe_combine_dual_residual gather + top-K weighted sum back to token order,
  *                             fused with the FarSkip-Collective dual residual
  *
- * and around them: the backward of each step (moe_combine_dual_residual_backward,
+ * (moe_route_dispatch runs the first three as one call, in one kernel when the
+ * batch fits) and around them: the backward of each step (moe_combine_dual_residual_backward,
  * moe_dispatch_backward, moe_route_topk_backward), the combine over FP8 expert
  * outputs (moe_combine_fp8_dual_residual), the routing weights in dispatched
  * order (moe_dispatch_route_weights), a sigmoid / selection-bias /
@@ -371,6 +372,51 @@ MOE_API int moe_dispatch_layout_static(const int32_t *topk_idx, int S, int E, in
                                        int token_padding, int32_t *counts, int32_t *offsets,
                                        int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src,
                                        int64_t cap, int32_t *status, void *stream);
+
+/*
+ * moe_route_dispatch: moe_route_topk, moe_dispatch_layout and moe_dispatch in
+ * one call -- router top-K gating ([pplx] Introduction), the padded
+ * expert-contiguous layout ([pplx] Portable Kernels, Dispatch; [moonep] core
+ * API example, tuning parameters) and the row scatter, optionally FP8
+ * ([pplx] Dispatch; [deepep] Technical overview).  Every output is exactly
+ * what the three calls would write (same router, same stable counting sort,
+ * same FP8 arithmetic):
+ *   topk_idx, topk_w   as moe_route_topk
+ *   counts, offsets, rank_offsets, slot_of, row_src   as moe_dispatch_layout
+ *                      on those ids (R, token_padding, cap)
+ *   xd, xs             as moe_dispatch of x (dtype, quant) with that slot_of
+ * The token rows x do not depend on the routing, so when the batch's share of
+ * each SM fits in shared memory (for example S <= 4144 tokens of H = 7168 bf16
+ * with FP8 on a 148-SM B200) the call is ONE cooperative kernel that reads and
+ * quantises x while it routes, keeps the rows in shared memory until their
+ * slots are known and then stores them; otherwise it launches the three
+ * separate kernels.  moe_route_dispatch_kernels tells which.
+ *
+ * workspace: device scratch of at least moe_route_dispatch_workspace(S, E, K)
+ *   bytes, 256-byte aligned, owned by the caller.  ALL of it must be zero
+ *   before the first call (the fused kernel keeps per-CTA arrival marks there,
+ *   past the part moe_dispatch_layout uses); every completed call leaves it
+ *   ready for the next one, whatever the sizes; after a MOE_STATUS_TIMEOUT
+ *   zero all of it again.  Do not modify it between calls; concurrent calls
+ *   need separate workspaces.  The same buffer also serves
+ *   moe_dispatch_layout (for the same or smaller S, E, K).
+ * Device status: the union of the three calls' bits, and MOE_STATUS_TIMEOUT
+ *   if a bounded wait of the fused kernel ran out.
+ * Host checks: the union of the three calls' checks.
+ */
+MOE_API size_t moe_route_dispatch_workspace(int S, int E, int K);
+MOE_API int moe_route_dispatch(const float *logits, const void *x, int dtype, int S, int H, int E, int K, int R,
+                               int token_padding, int quant, int32_t *topk_idx, float *topk_w, int32_t *counts,
+                               int32_t *offsets, int32_t *rank_offsets, int32_t *slot_of, int32_t *row_src,
+                               void *xd, float *xs, int64_t cap, void *workspace, size_t workspace_bytes,
+                               int32_t *status, void *stream);
+
+/*
+ * Kernels moe_route_dispatch launches for these sizes on the current device:
+ * 1 (the fused kernel) or 3 / 4 (router, layout in 1 or 2 kernels, dispatch).
+ * No launch happens.  Returns -1 on a CUDA error, 0 for invalid sizes.
+ */
+MOE_API int moe_route_dispatch_kernels(int S, int H, int E, int K, int dtype, int quant);
 
 /* Human-readable name of a return code (static string, host). */
 MOE_API const char *moe_error_string(int code);
