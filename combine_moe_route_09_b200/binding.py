@@ -46,6 +46,7 @@ SIGNATURES = {
     "moe_route_dispatch_kernels": (_I, [_I, _I, _I, _I, _I, _I]),
     "moe_route_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _L,
                                 _P, _Z, _P, _P]),
+    "moe_ep_plan": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_error_string": (ctypes.c_char_p, [_I]),
     "moe_capacity": (_L, [_I, _I, _I, _I]),
 }

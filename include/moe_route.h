@@ -418,6 +418,40 @@ MOE_API int moe_route_dispatch(const float *logits, const void *x, int dtype, in
  */
 MOE_API int moe_route_dispatch_kernels(int S, int H, int E, int K, int dtype, int quant);
 
+/* ------------------------------------------------------------------------ */
+/* Expert parallelism over W ranks (one GPU each).  Each rank routes its own  */
+/* tokens and builds its local layout with R = W (moe_route_topk,             */
+/* moe_dispatch_layout, P = 0): that layout is its send buffer, rank-major.   */
+/* The ranks exchange their per-expert counts (an all-gather of [E] int32),   */
+/* and each derives the same receive plan with moe_ep_plan; rows then move    */
+/* between ranks (NCCL point-to-point, one segment per (peer, expert)) and    */
+/* the combine runs on each source rank over its own send-order buffer.       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Receive plan of expert parallelism (host memory, host computation, no GPU).
+ * [pplx] Portable Kernels: experts in blocks of E/W per rank, a fixed region
+ * per (source rank, local expert) in the receiver's buffer; [pplx] Dispatch:
+ * the rows of one expert contiguous at the receiver; [moonep] core API
+ * example: Buffer(S, H, K, E, num_ep_ranks), token_padding.
+ *
+ *   counts         [W, E] int32 (host, read): counts[s][e] = pairs of source
+ *                  rank s routed to expert e (its layout's `counts`)
+ *   expert_offsets [E + 1] int32 (host, written): the padded offsets of the
+ *                  whole batch, rank-major -- exactly moe_dispatch_layout's
+ *                  `offsets` for all ranks' tokens taken in rank order
+ *   recv_offsets   [W, W, E/W] int32 (host, written): recv_offsets[d][s][j] is
+ *                  the first row, in rank d's receive buffer, of source rank
+ *                  s's rows of expert d*E/W + j (they follow in source order)
+ *   recv_rows      [W] int32 (host, written): rows of rank d's receive buffer
+ *                  (padding included)
+ * Returns MOE_OK, or MOE_ERR_INVALID_ARG for W < 1, E outside
+ * [1, MOE_MAX_EXPERTS], E % W != 0, token_padding < 0, a negative count, a
+ * total past 2^31 - 1 rows, or a NULL pointer.
+ */
+MOE_API int moe_ep_plan(const int32_t *counts, int W, int E, int token_padding, int32_t *expert_offsets,
+                        int32_t *recv_offsets, int32_t *recv_rows);
+
 /* Human-readable name of a return code (static string, host). */
 MOE_API const char *moe_error_string(int code);
 
