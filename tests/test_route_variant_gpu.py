@@ -98,3 +98,27 @@ def test_variant_empty_and_bad_args():
         K = kw.pop("K", 4)
         with pytest.raises(B.MoeError):
             B.moe_route_sigmoid_grouped(lg, K, **kw)
+
+
+@pytest.mark.parametrize("E,K,n_group,topk_group,use_bias,normalize,scale", [
+    (256, 8, 8, 4, True, True, 2.5),     # DeepSeek-V3-shaped
+    (64, 6, 4, 2, True, False, 1.0),
+    (96, 8, 1, 1, False, True, 1.0),
+    (40, 4, 8, 3, True, True, 0.5),      # groups of 5
+    (1024, 32, 32, 8, True, True, 1.0),  # largest E and K
+])
+def test_kernel_matches_fp64_reference(E, K, n_group, topk_group, use_bias, normalize, scale):
+    """The kernel against a reference that shares nothing with the oracle's exp:
+    scipy's fp64 sigmoid and library sorts with group masking, on logits spaced
+    far wider than fp32 rounding (so both precisions agree on every order).
+    Experts must be identical; weights within 4 fp32 ulp per term of the
+    normalising sum, (K + 4) * 4 * 2^-24 relative."""
+    from .test_oracle_route_variant import _grid_logits, _reference
+
+    rng = np.random.default_rng(E + K + 1)
+    logits = _grid_logits(rng, 200, E)
+    bias = (rng.permutation(E) * 0.0101).astype(np.float32) if use_bias else None
+    idx, w = _run(logits, K, bias, n_group, topk_group, normalize, scale)
+    ridx, rw = _reference(logits, K, bias, n_group, topk_group, normalize, scale)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=4 * 2.0 ** -24 * (K + 4), atol=0)

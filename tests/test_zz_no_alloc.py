@@ -5,23 +5,29 @@ layout (a framework or plugin that owns all device memory up front, or a
 latency-critical loop that cannot afford cudaMalloc's device synchronisation):
 its scratch is a fixed array inside the library instead of a caller-supplied
 workspace.  These tests call it through the C ABI and require outputs identical
-to moe_dispatch_layout's (the layout is integer work: bit-exact), on two calls
-in a row, so that leftovers of one call in the shared array cannot change the
-next.  The file is named to be collected last.
+to the CPU oracle's layout and to moe_dispatch_layout's (the layout is integer
+work: bit-exact), on two calls in a row, so that leftovers of one call in the
+shared array cannot change the next.  The cases cover every layout kernel:
+the single-cluster one (no scratch), the cooperative one (the grid-barrier
+header) and the histogram + slots pair (the arrival ticket and the per-tile
+histograms, all in the shared array).  The file is named to be collected last.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from combine_moe_route_09_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
 
-CASES = [  # S, E, K, R, token_padding
-    (4096, 256, 8, 8, 0),     # DeepSeek-V3-shaped prefill
-    (16384, 64, 8, 8, 128),   # imbalanced 16B-A3B-style, padded
-    (4099, 384, 8, 4, 128),   # ragged tail, E = 384
-    (3, 8, 2, 2, 4),          # a few tokens
+CASES = [  # S, E, K, R, token_padding, kernels moe_dispatch_layout launches
+    (4096, 256, 8, 8, 0, 1),      # DeepSeek-V3-shaped prefill: one cluster, no scratch
+    (16384, 64, 8, 8, 128, 1),    # imbalanced 16B-A3B-style, padded: cooperative grid
+    (4099, 384, 8, 4, 128, 1),    # ragged tail, E = 384
+    (3, 8, 2, 2, 4, 1),           # a few tokens
+    (8192, 1024, 32, 8, 16, 2),   # 128 tiles x 1024 experts: histogram + slots kernels
+    (32768, 1024, 8, 8, 0, 2),    # the same path with K = 8
 ]
 
 
@@ -38,15 +44,20 @@ def _assert_same(a: B.Layout, b: B.Layout):
         assert torch.equal(getattr(a, k), getattr(b, k)), k
 
 
-@pytest.mark.parametrize("S,E,K,R,P", CASES)
-def test_static_layout_matches_workspace_layout_twice(S, E, K, R, P):
+@pytest.mark.parametrize("S,E,K,R,P,kernels", CASES)
+def test_static_layout_matches_oracle_and_workspace_layout_twice(S, E, K, R, P, kernels):
+    assert B.moe_dispatch_layout_workspace(S, E, K) <= B.MOE_STATIC_LAYOUT_SCRATCH_BYTES
+    assert B.moe_dispatch_layout_kernels(S, E, K) == kernels
     idx = _routing(S, E, K, seed=S + E)
+    ref_o = oracle.layout(idx.cpu().numpy(), E, R, P)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ref = B.moe_dispatch_layout(idx, E, R, P, status=status)
     for _ in range(2):
         got = B.moe_dispatch_layout_static(idx, E, R, P, status=status)
         torch.cuda.synchronize()
         _assert_same(got, ref)
+        for k in ("counts", "offsets", "rank_offsets", "slot_of", "row_src"):
+            np.testing.assert_array_equal(getattr(got, k).cpu().numpy(), ref_o[k], err_msg=k)
     assert status.item() == 0
 
 
