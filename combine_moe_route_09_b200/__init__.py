@@ -10,6 +10,10 @@ The four calls of one MoE routing pass, each a C-ABI entry point of
 * :func:`moe_combine_dual_residual` — weighted gather with the FarSkip
   dual-residual epilogue
 
+:func:`moe_route_dispatch` runs the first three as one call (one kernel when
+that is faster); :class:`buffer.MoeBuffer` preallocates one pass;
+:mod:`ep` runs the pass with experts spread over several GPUs.
+
 Importing the package does not load the library; the first call does, and
 raises if it is missing.
 """
@@ -43,6 +47,9 @@ from .binding import (  # noqa: F401
     moe_dispatch_layout_static,
     moe_dispatch_layout_workspace,
     moe_dispatch_route_weights,
+    moe_route_dispatch,
+    moe_route_dispatch_kernels,
+    moe_route_dispatch_workspace,
     moe_route_sigmoid_grouped,
     moe_route_topk,
     moe_route_topk_backward,
