@@ -191,28 +191,32 @@ class MoeBuffer:
         return g
 
     def _choose_plan(self, calls: int = 10, reps: int = 5):
-        """Times route + layout + dispatch both ways -- the fused kernel and the
-        separate kernels -- on synthetic inputs of this buffer's shapes, each as a
-        CUDA graph of `calls` back-to-back calls, and keeps the faster (median of
-        `reps`).  Both plans write identical outputs; only the speed differs."""
+        """Times whole steps both ways -- route + layout + dispatch as the fused
+        kernel or as the separate kernels, then the combine -- on synthetic inputs
+        of this buffer's shapes (expert outputs, shared and residual rows drawn
+        for the purpose and freed after), each as a CUDA graph of `calls` steps,
+        and keeps the faster plan (median of `reps`).  The combine is timed too
+        because the plan changes what it finds in L2.  Both plans write identical
+        outputs; only the speed differs."""
         dev = self.device
         gen = torch.Generator(device=dev).manual_seed(0)
         logits = torch.randn((self.S, self.E), generator=gen, device=dev)
         x = torch.randn((self.S, self.H), generator=gen, device=dev).to(self.dtype)
+        y = torch.randn((self.cap, self.H), generator=gen, device=dev).to(self.dtype)
+        sh = torch.randn((self.S, self.H), generator=gen, device=dev).to(self.dtype)
+        rs = torch.randn((self.S, self.H), generator=gen, device=dev).to(self.dtype)
         side = torch.cuda.Stream(dev)
         times = {}
         with torch.cuda.device(dev):
             for fused in (True, False):
                 self.fused = fused
-                run = (lambda: self.route_dispatch(logits, x)) if fused else \
-                    (lambda: (self.route(logits), self.plan(), self.dispatch(x)))
-                run()
+                self.step(logits, x, y, sh, rs)
                 torch.cuda.synchronize(dev)
                 g = torch.cuda.CUDAGraph()
                 side.wait_stream(torch.cuda.current_stream(dev))
                 with torch.cuda.graph(g, stream=side):
                     for _ in range(calls):
-                        run()
+                        self.step(logits, x, y, sh, rs)
                 g.replay()
                 torch.cuda.synchronize(dev)
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -225,6 +229,7 @@ class MoeBuffer:
                     ts.append(a.elapsed_time(b) * 1e3 / calls)
                 del g
                 times["fused" if fused else "separate"] = sorted(ts)[len(ts) // 2]
+        del logits, x, y, sh, rs
         self.fused = times["fused"] <= times["separate"]
         self.plan_timings_us = times
         self._seen.clear()
