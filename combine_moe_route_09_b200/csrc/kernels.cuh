@@ -25,8 +25,9 @@ inline size_t layout_workspace_bytes(int S, int E, int K) {
     return LT_HEADER + ((hist + 255) / 256) * 256;
 }
 
-// Fused route + layout + dispatch: scratch header, then [RD_MAX_CTAS][E rounded up to 4] int32.
-constexpr size_t RD_HEADER_BYTES = LT_HEADER;
+// Fused route + layout + dispatch.  Its workspace is the layout's workspace,
+// then (256-byte aligned) the arrival marks [RD_MAX_CTAS] u32 and the per-CTA
+// histogram rows [RD_MAX_CTAS][E rounded up to 8] u16.
 constexpr int RD_MAX_CTAS = 512;
 size_t route_dispatch_workspace_bytes(int S, int E, int K);
 // Kernels moe_route_dispatch launches for these sizes on the current device (1 fused, else 3 or 4; -1: CUDA error).

@@ -12,20 +12,27 @@
 // moe_dispatch_layout and moe_dispatch (the same per-row router, the same
 // stable counting sort, the same FP8 arithmetic); what changes is when the
 // bytes move.  The token rows x do not depend on the routing, so they are read
-// and quantised while the router runs, and kept in shared memory until their
+// (and quantised) while the router runs, and kept in shared memory until their
 // slots are known; the rows then leave as TMA bulk stores.  One CTA per SM,
 // all co-resident (cooperative launch); CTA b owns the contiguous tokens
-// [S*b/G, S*(b+1)/G).
+// [S*b/G, S*(b+1)/G).  The host takes this kernel only for small shares
+// (FP8: at most RD_FP8_MAX_TOKENS tokens per CTA), where the exchange and the
+// quantiser cost less than the separate kernels' launches and round trips.
 //
 // Warp roles:
-//   producer (warp 0)  bulk-loads each token's x row into the resident region
-//   quantisers (1..8)  FP8 only: turn token j's raw row into its resident
-//                      slot j (codes, then the block scales), in token order
-//   routers (9..16)    route the CTA's tokens (one warp per token), rank the
-//                      CTA's (token, k) pairs by expert, publish the CTA's
-//                      expert histogram, take part in the one grid barrier,
-//                      compute the offsets and slots, then issue the K bulk
-//                      stores of each resident token as soon as it is ready
+//   producer (warp 0)    waits until the routing warps hold their first logits,
+//                        then bulk-loads each token's x row into the resident
+//                        region (at most `inflight` rows in flight)
+//   all 16 other warps   route the CTA's tokens (one warp per token); the
+//                        experts and weights go to shared memory
+//   quantisers (1..8)    FP8 only, in groups of P warps per token: turn token
+//                        j's raw row into its resident slot j (codes, then the
+//                        block scales)
+//   routers (9..16)      rank the CTA's (token, k) pairs by expert, publish
+//                        the CTA's histogram row and arrival mark, wait for
+//                        every CTA's mark, compute the offsets and slots,
+//                        write the layout and gating outputs, then issue the K
+//                        bulk stores of each resident token once it is final
 //
 // The resident region has Qs slots of qrow bytes (FP8: codes + scales of one
 // token).  A raw row needs rho slots (bf16 input: 2, fp32: 4).  Raw rows are
@@ -35,9 +42,11 @@
 // is written only once token j's raw row is in registers, and every raw row j
 // lies at slots >= j.  With Qs = M + rho - 1 every token of a CTA with M
 // tokens finds a window.  Before a raw row is loaded into a window, the last
-// token whose raw row covered that window must be done (its mbarrier).
+// token whose raw row covered that window must be done (its mbarrier); before
+// a quantiser group writes slot j, the token whose raw row last covered slot
+// j must be done too (the groups run tokens out of order).
 //
-// Every wait is bounded (mbarriers and the grid barrier); a timeout sets
+// Every wait is bounded (mbarriers and the arrival-mark poll); a timeout sets
 // MOE_STATUS_TIMEOUT and every role leaves its loop; loads in flight are
 // waited for (bounded) before the CTA exits.
 #include "common.cuh"
