@@ -134,6 +134,36 @@ def test_full_pass_as_benchmarked(case):
     assert int(buf.workspace[:8].sum().item()) == 0  # arrival ticket and barrier count back at zero
 
 
+def test_both_step_plans_give_the_pass(case):
+    """MoeBuffer.step with route + layout + dispatch in the fused kernel (where it
+    applies) and with the separate kernels: the same pass both times."""
+    w, inp, ref = case
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    q = B.MOE_QUANT_FP8_E4M3_B128 if w.quant == "fp8" else B.MOE_QUANT_NONE
+    applies = B.moe_route_dispatch_kernels(w.S, w.H, w.E, w.K, dt, q) == 1
+    buf = MoeBuffer(w.S, w.H, w.K, w.E, w.R, w.P, dtype=dt, fp8=w.quant == "fp8", fused=applies)
+    args = [dev(inp["logits"]), dev(inp["x"]), dev(inp["y"])]
+    if w.fused:
+        args += [dev(inp["shared"]), dev(inp["residual"])]
+    weight_slack = 2e-5 * abs_weighted_sum(inp["y"], ref["lay"]["slot_of"], ref["w"])
+    valid = ref["lay"]["row_src"] >= 0
+    for fused in ([True, False] if applies else [False]):
+        buf.fused = fused
+        assert buf.kernels_per_step == (2 if fused else 3 + B.moe_dispatch_layout_kernels(w.S, w.E, w.K))
+        buf.layout.slot_of.fill_(-7)
+        buf.topk_idx.fill_(-7)
+        buf.out.zero_()
+        buf.step(*args)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(buf.topk_idx), ref["idx"])
+        _check_layout(buf.layout, ref["lay"])
+        np.testing.assert_array_equal(host(buf.xd)[valid], ref["xd"][valid])
+        if w.quant == "fp8":
+            np.testing.assert_array_equal(host(buf.xs)[valid], ref["xs"][valid])
+        assert_act_close(host(buf.out), ref["out"], "residual_out", extra_abs=weight_slack)
+        assert buf.read_status() == 0
+
+
 def test_captured_step_replays_the_pass(case):
     """One step captured in a CUDA graph and replayed twice gives the oracle's pass."""
     w, inp, ref = case

@@ -6,7 +6,8 @@ bit for bit, with the three separate entry points on the same inputs.  The
 cases cover the workloads that run as one fused kernel, the ragged and
 maximum shares per CTA, the fallback to separate kernels, scale rows that are
 not whole 16-byte units, two quantisation passes, fp32 input, K = E, padding,
-a capacity smaller than the layout, heavy ties and graph replay.
+a capacity smaller than the layout, heavy ties, graph replay and a workspace
+shared with moe_dispatch_layout.
 """
 import numpy as np
 import pytest
@@ -233,3 +234,60 @@ def test_repeated_calls_and_graph_replay_with_new_inputs():
     _assert_oracle(w2, lg2, x2, (idx, wt, lay, xd, xs))
     assert status.item() == 0
     assert int(ws[:8].sum().item()) == 0  # grid-barrier count back at zero
+
+
+def test_one_workspace_shared_with_the_layout_entry_point():
+    """moe_route_dispatch (fused) and moe_dispatch_layout take turns on one
+    workspace, eagerly and inside a replayed graph; every call gives the
+    separate kernels' results and leaves the workspace ready."""
+    w = _wl(300, 1024, 256, 8, 8, 0, "bf16", "fp8", seed=31)
+    assert B.moe_route_dispatch_kernels(w.S, w.H, w.E, w.K, torch.bfloat16, _qcode(w)) == 1
+    lg, x = synth.logits(w), synth.activations(w)
+    dl, dx = dev(lg), dev(x)
+    cap = B.moe_capacity(w.S, w.E, w.K, w.P)
+    ref = _separate(w, dl, dx)
+    need = max(B.moe_route_dispatch_workspace(w.S, w.E, w.K), B.moe_dispatch_layout_workspace(w.S, w.E, w.K))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    idx = torch.empty((w.S, w.K), **i32)
+    wt = torch.empty((w.S, w.K), dtype=torch.float32, device="cuda")
+    lay = B.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32), torch.empty(w.R + 1, **i32),
+                   torch.empty((w.S, w.K), **i32), torch.empty(cap, **i32), cap)
+    xd, xs = _sentinels(w, cap)
+
+    def reset():
+        idx.fill_(-3)
+        wt.fill_(-3.0)
+        for k in LAYOUT_KEYS:
+            getattr(lay, k).fill_(-3)
+
+    def rd():
+        B.moe_route_dispatch(dl, dx, w.K, w.R, w.P, _qcode(w), cap, topk_idx=idx, topk_w=wt, layout=lay, xd=xd,
+                             xs=xs, workspace=ws, status=status)
+
+    def lay_only():
+        B.moe_dispatch_layout(ref[0], w.E, w.R, w.P, cap, out=lay, workspace=ws, status=status)
+
+    def check(full):
+        torch.cuda.synchronize()
+        if full:
+            assert torch.equal(idx, ref[0]) and torch.equal(wt, ref[1])
+            assert torch.equal(xd.view(torch.uint8), ref[3].view(torch.uint8)) and torch.equal(xs, ref[4])
+        for k in LAYOUT_KEYS:
+            assert torch.equal(getattr(lay, k), getattr(ref[2], k)), k
+
+    for f, full in [(rd, True), (lay_only, False), (lay_only, False), (rd, True), (rd, True), (lay_only, False),
+                    (rd, True)]:
+        reset()
+        f()
+        check(full)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lay_only()
+        rd()
+    for _ in range(3):
+        reset()
+        g.replay()
+        check(True)
+    assert status.item() == 0
