@@ -12,30 +12,34 @@
 // Persistent kernel on the same pipeline as the forward combine: a producer
 // warp bulk-loads, per (token, chunk) item, the K gathered y chunks, the g
 // chunk and the gn chunk into a 2-stage ring (cp.async.bulk, mbarriers, no
-// multicast); 4 consumer warps hold one 16-byte unit per thread.  Each CTA
-// takes whole tokens, so grad_w needs no atomics: per item every warp reduces
-// its dot-product partials with a fixed xor tree and lane k keeps pair k's
-// running sum; at the token's last chunk the four warps' sums are added in
-// warp order.  The reduction barrier there is an AND-barrier, so a timed-out
-// wait makes all consumer warps leave together.
+// multicast); W consumer warps (4, or 16 for rows longer than 8 KB) hold one
+// 16-byte unit per thread.  Each CTA takes whole tokens, so grad_w needs no
+// atomics: per item every warp reduces its dot-product partials with a fixed
+// xor tree and lane k keeps pair k's running sum; at the token's last chunk the
+// W warps' sums are added in warp order.  The reduction barrier there is an
+// AND-barrier, so a timed-out wait makes all consumer warps leave together.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tma.cuh"
 
 namespace moe {
 
-// 4 consumer warps with 2 KB chunks in 2 stages (about 42 KB a CTA, 5 CTAs an SM
-// at K = 8).  A sweep of 4 to 16 consumer warps, 2 to 4 stages and 1 to 5 CTAs an
-// SM found no setting faster on every shape: 16 warps (8 KB chunks) took 195 us
-// instead of 205 us on 4096 x 7168 but 41 us instead of 19.5 us on 4096 x 768;
-// 6 warps took 211 us instead of 230 us on 16384 x 2048 and 209 us on 4096 x 7168.
+// 2 stages.  Rows of at most 8 KB: 4 consumer warps with 2 KB chunks (about 42 KB
+// a CTA, 5 CTAs an SM at K = 8).  Longer rows: 16 warps with 8 KB chunks (one
+// CTA an SM).  A sweep of 4 to 16 consumer warps, 2 to 4 stages and 1 to 5 CTAs
+// an SM found no single setting faster on every shape: 16 warps took 195 us
+// instead of 205 us on 4096 x 7168 (and the backward step 270.9 against 282.4 us)
+// but 41 us instead of 19.5 us on 4096 x 768, and gained nothing on 16384 x 2048.
 constexpr int BW_STAGES = 2;
-constexpr int BW_CONSUMER_WARPS = 4;
-constexpr int BW_CONSUMERS = BW_CONSUMER_WARPS * 32;
-constexpr int BW_THREADS = BW_CONSUMERS + 32;
-constexpr int BW_MAX_CHUNK = BW_CONSUMERS * 16;
 constexpr int BW_HDR = 384;  // per stage: valid mask, the token's K weights (at 4), K slots (at 132)
-constexpr int BW_SMEM_BUDGET = 100 * 1024;
+constexpr int BW_LONG_ROW = 8192;  // bytes: longer rows take 16 consumer warps, the others 4
+template <int W>
+struct BwShape {
+    static constexpr int CONSUMERS = W * 32;
+    static constexpr int THREADS = CONSUMERS + 32;  // + the producer warp
+    static constexpr int MAX_CHUNK = CONSUMERS * 16;
+    static constexpr int SMEM_BUDGET = W > 4 ? 200 * 1024 : 100 * 1024;  // ring bytes per CTA
+};
 
 struct CombineBwdArgs {
     const uint8_t *g, *gn, *y;
@@ -78,8 +82,8 @@ struct BVec<true> {
     }
 };
 
-template <bool F32, bool HAS_GN, bool HAS_SKIP>
-__global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBwdArgs a) {
+template <int W, bool F32, bool HAS_GN, bool HAS_SKIP>
+__global__ void __launch_bounds__(BwShape<W>::THREADS) combine_bwd_kernel(const CombineBwdArgs a) {
     using V = BVec<F32>;
     constexpr int N = V::N;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     if (tid == 0) {
         for (int s = 0; s < BW_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), BW_CONSUMER_WARPS);
+            mbar_init(empty_bar(s), W);
         }
         fence_mbar_init();
     }
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     const int t_last = (int)((long long)a.S * (blockIdx.x + 1) / gridDim.x);
     const long long first = (long long)t_first * a.nchunks, last = (long long)t_last * a.nchunks;
 
-    if (warp == BW_CONSUMER_WARPS) {
+    if (warp == W) {
         // ------------------------------- producer -------------------------------
         int t_cur = -1, cur = -1, nxt = -1;
         float cur_w = 0.f, nxt_w = 0.f;
@@ -229,15 +233,15 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
             if (lane == 0) mbar_arrive(empty_bar(s));
         }
         if (c == a.nchunks - 1) {
-            // token end: add the four warps' sums in warp order
+            // token end: add the W warps' sums in warp order
             const int par = ntok & 1;
-            if (lane < K) wsum[(par * BW_CONSUMER_WARPS + warp) * 32 + lane] = run;
-            if (!named_bar_and(1, BW_CONSUMERS, !failed)) break;
+            if (lane < K) wsum[(par * W + warp) * 32 + lane] = run;
+            if (!named_bar_and(1, BwShape<W>::CONSUMERS, !failed)) break;
             if (warp == 0 && lane < K) {
                 float sum = 0.f;
 #pragma unroll
-                for (int ww = 0; ww < BW_CONSUMER_WARPS; ++ww)
-                    sum = __fadd_rn(sum, wsum[(par * BW_CONSUMER_WARPS + ww) * 32 + lane]);
+                for (int ww = 0; ww < W; ++ww)
+                    sum = __fadd_rn(sum, wsum[(par * W + ww) * 32 + lane]);
                 a.grad_w[(size_t)t * K + lane] = sum;
             }
             run = 0.f;
@@ -246,27 +250,31 @@ __global__ void __launch_bounds__(BW_THREADS) combine_bwd_kernel(const CombineBw
     }
 }
 
-template <bool F32, bool GN, bool SKIP>
-static cudaError_t launch_bwd(const CombineBwdArgs &a, cudaStream_t st) {
-    auto kern = combine_bwd_kernel<F32, GN, SKIP>;
+template <int W, bool F32, bool GN, bool SKIP>
+static cudaError_t launch_bwd(CombineBwdArgs a, cudaStream_t st) {
+    auto kern = combine_bwd_kernel<W, F32, GN, SKIP>;
+    int chunk = BwShape<W>::MAX_CHUNK;
+    while (chunk > 256 && BW_STAGES * (BW_HDR + (a.K + 2) * chunk) > BwShape<W>::SMEM_BUDGET) chunk >>= 1;
+    a.chunk = chunk < a.row_bytes ? chunk : a.row_bytes;
+    a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
     const size_t smem = (size_t)BW_STAGES * (BW_HDR + (a.K + 2) * a.chunk) + 2 * BW_STAGES * 8 +
-                        2 * BW_CONSUMER_WARPS * 32 * sizeof(float);
+                        2 * W * 32 * sizeof(float);
     static KernelSlots<decltype(kern)> slots;
     int sms = 0, per_sm = 0;
-    cudaError_t e = slots.prepare(kern, BW_THREADS, smem, &sms, &per_sm);
+    cudaError_t e = slots.prepare(kern, BwShape<W>::THREADS, smem, &sms, &per_sm);
     if (e != cudaSuccess) return e;
     long long grid = (long long)sms * per_sm;
     if (grid > a.S) grid = a.S;
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(BW_THREADS), smem, st, a);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(BwShape<W>::THREADS), smem, st, a);
 }
 
-template <bool F32>
+template <int W, bool F32>
 static cudaError_t launch_bwd_dt(const CombineBwdArgs &a, cudaStream_t st) {
     const bool gn = a.gn, skip = a.grad_skip;
-    if (gn && skip) return launch_bwd<F32, true, true>(a, st);
-    if (gn) return launch_bwd<F32, true, false>(a, st);
-    if (skip) return launch_bwd<F32, false, true>(a, st);
-    return launch_bwd<F32, false, false>(a, st);
+    if (gn && skip) return launch_bwd<W, F32, true, true>(a, st);
+    if (gn) return launch_bwd<W, F32, true, false>(a, st);
+    if (skip) return launch_bwd<W, F32, false, true>(a, st);
+    return launch_bwd<W, F32, false, false>(a, st);
 }
 
 cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y, int dtype, int S, int H,
@@ -289,11 +297,8 @@ cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y
     a.S = S;
     a.K = K;
     a.row_bytes = H * (f32 ? 4 : 2);
-    int chunk = BW_MAX_CHUNK;
-    while (chunk > 256 && BW_STAGES * (BW_HDR + (K + 2) * chunk) > BW_SMEM_BUDGET) chunk >>= 1;
-    a.chunk = chunk < a.row_bytes ? chunk : a.row_bytes;
-    a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
-    return f32 ? launch_bwd_dt<true>(a, st) : launch_bwd_dt<false>(a, st);
+    if (a.row_bytes > BW_LONG_ROW) return f32 ? launch_bwd_dt<16, true>(a, st) : launch_bwd_dt<16, false>(a, st);
+    return f32 ? launch_bwd_dt<4, true>(a, st) : launch_bwd_dt<4, false>(a, st);
 }
 
 }  // namespace moe
