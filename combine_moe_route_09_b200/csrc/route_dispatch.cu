@@ -27,7 +27,8 @@
 //                        experts and weights go to shared memory
 //   quantisers (1..8)    FP8 only, in groups of P warps per token: turn token
 //                        j's raw row into its resident slot j (codes, then the
-//                        block scales)
+//                        block scales); with at most 2 tokens per CTA they
+//                        start once the routers have published the CTA's counts
 //   routers (9..16)      rank the CTA's (token, k) pairs by expert, publish
 //                        the CTA's histogram row and arrival mark, wait for
 //                        every CTA's mark, compute the offsets and slots,
@@ -75,6 +76,7 @@ constexpr int RD_FP8_MAX_TOKENS = 4;
 constexpr int RD_BAR_R = 2;                  // named barrier of the routers (id 1 is not used)
 constexpr int RD_BAR_ROUTED = 3;             // quantisers arrive, routers wait: routing complete
 constexpr int RD_BAR_GROUP0 = 4;             // 4 .. 11: quantiser groups
+constexpr int RD_BAR_PUBLISHED = 12;         // routers arrive once the CTA's counts are out, quantisers wait
 constexpr long long RD_INFLIGHT_BYTES = 64 * 1024;  // token-row bytes a CTA keeps in flight
 
 struct RdArgs {
@@ -97,6 +99,7 @@ struct RdArgs {
     int Ep;          // E rounded up to a multiple of 8 (hist row stride: 16-byte rows of uint16)
     int inflight;    // raw rows a CTA keeps in flight at most
     int qgroup;      // quantiser warps per token (1, 2, 4 or 8)
+    int qdelay;      // FP8: the quantisers start once the routers have published the CTA's counts
     int M;           // tokens per CTA at most
     int qrow;        // bytes of one resident slot (multiple of 16)
     int rho;         // slots covered by one raw row
@@ -266,6 +269,10 @@ __global__ void __launch_bounds__(RD_THREADS, 1) route_dispatch_kernel(const RdA
         // last iteration.  Before writing slot j the group waits for the token
         // whose raw row last covered that slot.
         if (!a.quant) return;
+        // With few tokens per CTA the quantisers are off the critical path, which
+        // runs through the routers' ranking and the exchange: keeping the SM's
+        // issue slots for the routers until their counts are published shortens it.
+        if (a.qdelay) named_bar(RD_BAR_PUBLISHED, RD_QT + RD_RT);
         const int qw = warp - 1;
         const int P = a.qgroup, NG = RD_QUANT_WARPS / P;
         const int g = qw / P, gm = qw - g * P;
@@ -413,6 +420,7 @@ __global__ void __launch_bounds__(RD_THREADS, 1) route_dispatch_kernel(const RdA
     named_bar(RD_BAR_R, RD_RT);
     const unsigned epoch = s_epoch;
     if (rt == 0) *(volatile unsigned *)&a.arrived[b] = epoch;
+    if (a.quant && a.qdelay) named_bar_arrive(RD_BAR_PUBLISHED, RD_QT + RD_RT);  // the quantisers may start
     bool layout_ok = true;
     {
         const unsigned long long t_start = globaltimer();
@@ -667,6 +675,7 @@ static cudaError_t rd_plan(int S, int H, int E, int K, int R, int P, int dtype, 
     a->quant = quant ? 1 : 0;
     a->Ep = rd_row(E);
     a->qgroup = M >= 8 ? 1 : (M >= 4 ? 2 : (M >= 2 ? 4 : 8));
+    a->qdelay = quant && M <= 2 ? 1 : 0;
     a->inflight = (int)(RD_INFLIGHT_BYTES / row_bytes > 1 ? RD_INFLIGHT_BYTES / row_bytes : 1);
     a->M = M;
     a->qrow = qrow;
