@@ -12,8 +12,8 @@
 // Persistent kernel on the same pipeline as the forward combine: a producer
 // warp bulk-loads, per (token, chunk) item, the K gathered y chunks, the g
 // chunk and the gn chunk into a 2-stage ring (cp.async.bulk, mbarriers, no
-// multicast); W consumer warps (4, or 16 for rows longer than 8 KB) hold one
-// 16-byte unit per thread.  Each CTA takes whole tokens, so grad_w needs no
+// multicast); W consumer warps (4 for rows up to 2 KB, 6 up to 8 KB, 16 for
+// longer rows) hold one 16-byte unit per thread.  Each CTA takes whole tokens, so grad_w needs no
 // atomics: per item every warp reduces its dot-product partials with a fixed
 // xor tree and lane k keeps pair k's running sum; at the token's last chunk the
 // W warps' sums are added in warp order.  The reduction barrier there is an
@@ -24,15 +24,18 @@
 
 namespace moe {
 
-// 2 stages.  Rows of at most 8 KB: 4 consumer warps with 2 KB chunks (about 42 KB
-// a CTA, 5 CTAs an SM at K = 8).  Longer rows: 16 warps with 8 KB chunks (one
-// CTA an SM).  A sweep of 4 to 16 consumer warps, 2 to 4 stages and 1 to 5 CTAs
-// an SM found no single setting faster on every shape: 16 warps took 195 us
-// instead of 205 us on 4096 x 7168 (and the backward step 270.9 against 282.4 us)
-// but 41 us instead of 19.5 us on 4096 x 768, and gained nothing on 16384 x 2048.
+// 2 stages.  Rows of at most 2 KB: 4 consumer warps with 2 KB chunks (about 42 KB
+// a CTA, 5 CTAs an SM at K = 8).  Rows of at most 8 KB: 6 warps with 3 KB chunks
+// (3 CTAs an SM).  Longer rows: 16 warps with 8 KB chunks (one CTA an SM).  A
+// sweep of 4 to 16 consumer warps, 2 to 4 stages and 1 to 5 CTAs an SM found no
+// single setting faster on every shape.  In the graph-replayed backward step
+// (combine, dispatch and router backward): 16 warps took 4096 x 7168 from 282.4
+// to 270.9 us, 6 warps took 16384 x 2048 from 357.9 to 311.1 us (10 warps:
+// 311.2 us), while 4096 x 768 rows ran 19.5 us with 4 warps against 41 us with 16.
 constexpr int BW_STAGES = 2;
 constexpr int BW_HDR = 384;  // per stage: valid mask, the token's K weights (at 4), K slots (at 132)
-constexpr int BW_LONG_ROW = 8192;  // bytes: longer rows take 16 consumer warps, the others 4
+constexpr int BW_SHORT_ROW = 2048;  // bytes: rows up to this take 4 consumer warps
+constexpr int BW_LONG_ROW = 8192;   // bytes: rows up to this take 6 consumer warps, longer rows 16
 template <int W>
 struct BwShape {
     static constexpr int CONSUMERS = W * 32;
@@ -298,6 +301,7 @@ cudaError_t launch_combine_backward(const void *g, const void *gn, const void *y
     a.K = K;
     a.row_bytes = H * (f32 ? 4 : 2);
     if (a.row_bytes > BW_LONG_ROW) return f32 ? launch_bwd_dt<16, true>(a, st) : launch_bwd_dt<16, false>(a, st);
+    if (a.row_bytes > BW_SHORT_ROW) return f32 ? launch_bwd_dt<6, true>(a, st) : launch_bwd_dt<6, false>(a, st);
     return f32 ? launch_bwd_dt<4, true>(a, st) : launch_bwd_dt<4, false>(a, st);
 }
 

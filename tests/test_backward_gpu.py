@@ -3,7 +3,7 @@
 Tolerances: grad_y, grad_skip and the dispatch backward use the same fp32
 operations in the same order as the oracle (<= 1 bf16 ulp, or 1e-5 relative
 for fp32).  grad_w is an fp32 sum of H products in a fixed order (a thread's
-8 or 4 products, a 32-lane xor tree, the row's chunks, then the 4 or 16
+8 or 4 products, a 32-lane xor tree, the row's chunks, then the 4, 6 or 16
 consumer warps in order): a leaf passes at most 8 + 5 + chunks + warps
 roundings, 31 for the shapes here, so its error against the oracle's fp64 sum
 is at most about 32 * 2^-24 * sum_h |y_h g_h|.
@@ -44,6 +44,7 @@ CASES = [
     synth.WORKLOADS["5"].replace(S=3000),
     synth.WORKLOADS["4"].replace(S=500, H=4608),             # rows of 9 KB: 16 warps, a ragged second chunk
     synth.WORKLOADS["4"].replace(S=300, H=2304, dtype="f32"),  # fp32 rows of 9 KB
+    synth.WORKLOADS["5"].replace(S=700, H=1536, dtype="f32"),  # fp32 rows of 6 KB: 6 warps, 3 KB chunks
     synth.Workload("bwd_ragged", 777, 264, 40, 5, 4, 3, "bf16", "none", True, seed=31),
     synth.Workload("bwd_k17_f32", 301, 260, 17, 17, 17, 1, "f32", "none", True, seed=32),
 ]
