@@ -17,7 +17,7 @@
 //                   valid slot, plus the shared_out and residual chunks, into
 //                   a ring of STAGES shared-memory stages.  No tensor maps,
 //                   no multicast.
-//   8 consumer warps per item: one 16-byte unit per thread; acc = fma(w_k, y_k,
+//   6 or 8 consumer warps per item: one 16-byte unit per thread; acc = fma(w_k, y_k,
 //                   acc) in ascending k from shared memory, + shared, +
 //                   residual, round once, 16-byte stores of both streams;
 //                   then release the stage.
@@ -29,17 +29,24 @@
 
 namespace moe {
 
-// 8 consumer warps take 4 KB chunks (one 16-byte unit per thread) through a
-// 2-stage ring (82 KB per CTA with K = 8, two CTAs per SM).  On the
-// DeepSeek-V3-shaped prefill combine this ran 107.0 us against 110.9 us for 4
-// warps with 2 KB chunks in 4 stages; 3 or 4 stages of 4 KB, and 6 or 8
-// stages of smaller chunks, were slower.
+// W consumer warps take chunks of W * 512 bytes (one 16-byte unit per thread)
+// through a 2-stage ring.  Rows of 2 to 8 KB take 6 warps (3 KB chunks, three
+// CTAs per SM); the others take 8 warps (4 KB chunks, 82 KB per CTA with K = 8,
+// two CTAs per SM).  On the DeepSeek-V3-shaped prefill combine 8 warps ran
+// 107.0 us against 110.9 us for 4 warps with 2 KB chunks in 4 stages; 3 or 4
+// stages of 4 KB, and 6 or 8 stages of smaller chunks, were slower.  On the
+// 16384 x 2048 workload's 4 KB rows 6 warps took the step from 256.7 to
+// 252.7 us (10 or 12 warps: 254.8 us); on rows of at most 2 KB, 4 warps, fast
+// alone, lost in the step.
 constexpr int CB_STAGES = 2;
-constexpr int CB_CONSUMER_WARPS = 8;
-constexpr int CB_CONSUMERS = CB_CONSUMER_WARPS * 32;
-constexpr int CB_THREADS = CB_CONSUMERS + 32;
-constexpr int CB_MAX_CHUNK = CB_CONSUMERS * 16;  // 4096 bytes: one 16-byte unit per consumer
 constexpr int CB_SMEM_BUDGET = 100 * 1024;
+constexpr int CB_MID_WARPS = 6;  // consumer warps for rows of 2 to 8 KB; 8 for the others
+template <int W>
+struct CbShape {
+    static constexpr int CONSUMERS = W * 32;
+    static constexpr int THREADS = CONSUMERS + 32;  // + the producer warp
+    static constexpr int MAX_CHUNK = CONSUMERS * 16;
+};
 
 template <bool F32>
 struct Vec;
@@ -82,14 +89,14 @@ struct CombineArgs {
     int64_t cap;
     int S, K;
     int row_bytes;  // H * element size, a multiple of 16
-    int chunk;      // bytes per work item, a multiple of 16, <= CB_MAX_CHUNK
+    int chunk;      // bytes per work item, a multiple of 16, <= CbShape<W>::MAX_CHUNK
     int nchunks;    // ceil(row_bytes / chunk)
 };
 
 constexpr int CB_HDR = 256;  // per-stage header: valid mask, then the token's K weights
 
-template <bool F32, bool HAS_SH, bool HAS_RS, bool HAS_RNR>
-__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a) {
+template <int W, bool F32, bool HAS_SH, bool HAS_RS, bool HAS_RNR>
+__global__ void __launch_bounds__(CbShape<W>::THREADS) combine_kernel(const CombineArgs a) {
     using V = Vec<F32>;
     constexpr int N = V::N;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -107,7 +114,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
     if (tid == 0) {
         for (int s = 0; s < CB_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), CB_CONSUMER_WARPS);
+            mbar_init(empty_bar(s), W);
         }
         fence_mbar_init();
     }
@@ -120,7 +127,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
     const long long nitems = (long long)a.S * a.nchunks;
     const long long first = nitems * blockIdx.x / gridDim.x;
     const long long last = nitems * (blockIdx.x + 1) / gridDim.x;
-    if (warp == CB_CONSUMER_WARPS) {
+    if (warp == W) {
         // ------------------------------- producer -------------------------------
         // Lane k holds the token's slot k and weight k, loaded one token ahead.
         int t_cur = -1, cur = -1, nxt = -1;
@@ -232,8 +239,9 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
     }
 }
 
+template <int W>
 static int combine_chunk(int K, int row_bytes) {
-    int chunk = CB_MAX_CHUNK;
+    int chunk = CbShape<W>::MAX_CHUNK;
     while (chunk > 256 && CB_STAGES * (CB_HDR + (K + 2) * chunk) > CB_SMEM_BUDGET) chunk >>= 1;
     return chunk < row_bytes ? chunk : row_bytes;
 }
@@ -242,28 +250,30 @@ static size_t combine_smem(int K, int chunk) {
     return (size_t)CB_STAGES * (CB_HDR + (K + 2) * chunk) + 2 * CB_STAGES * 8;
 }
 
-template <bool F32, bool SH, bool RS, bool RNR>
-static cudaError_t launch_cb(const CombineArgs &a, cudaStream_t st) {
-    auto kern = combine_kernel<F32, SH, RS, RNR>;
+template <int W, bool F32, bool SH, bool RS, bool RNR>
+static cudaError_t launch_cb(CombineArgs a, cudaStream_t st) {
+    auto kern = combine_kernel<W, F32, SH, RS, RNR>;
+    a.chunk = combine_chunk<W>(a.K, a.row_bytes);
+    a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
     const size_t smem = combine_smem(a.K, a.chunk);
     static KernelSlots<decltype(kern)> slots;
     int sms = 0, per_sm = 0;
-    cudaError_t e = slots.prepare(kern, CB_THREADS, smem, &sms, &per_sm);
+    cudaError_t e = slots.prepare(kern, CbShape<W>::THREADS, smem, &sms, &per_sm);
     if (e != cudaSuccess) return e;
     const long long nitems = (long long)a.S * a.nchunks;
     long long grid = (long long)sms * per_sm;
     if (grid > nitems) grid = nitems;
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(CB_THREADS), smem, st, a);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(CbShape<W>::THREADS), smem, st, a);
 }
 
-template <bool F32>
+template <int W, bool F32>
 static cudaError_t launch_cb_dt(const CombineArgs &a, cudaStream_t st) {
     const bool sh = a.shared_out, rs = a.residual, rnr = a.out_no_routed;
-    if (sh && rs && rnr) return launch_cb<F32, true, true, true>(a, st);
-    if (sh && rs) return launch_cb<F32, true, true, false>(a, st);
-    if (sh) return launch_cb<F32, true, false, false>(a, st);
-    if (rs) return launch_cb<F32, false, true, false>(a, st);
-    return launch_cb<F32, false, false, false>(a, st);
+    if (sh && rs && rnr) return launch_cb<W, F32, true, true, true>(a, st);
+    if (sh && rs) return launch_cb<W, F32, true, true, false>(a, st);
+    if (sh) return launch_cb<W, F32, true, false, false>(a, st);
+    if (rs) return launch_cb<W, F32, false, true, false>(a, st);
+    return launch_cb<W, F32, false, false, false>(a, st);
 }
 
 cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_t cap,
@@ -285,9 +295,9 @@ cudaError_t launch_combine(const void *y, int dtype, int S, int H, int K, int64_
     a.S = S;
     a.K = K;
     a.row_bytes = H * (f32 ? 4 : 2);
-    a.chunk = combine_chunk(K, a.row_bytes);
-    a.nchunks = (a.row_bytes + a.chunk - 1) / a.chunk;
-    return f32 ? launch_cb_dt<true>(a, st) : launch_cb_dt<false>(a, st);
+    if (a.row_bytes > 2048 && a.row_bytes <= 8192)
+        return f32 ? launch_cb_dt<CB_MID_WARPS, true>(a, st) : launch_cb_dt<CB_MID_WARPS, false>(a, st);
+    return f32 ? launch_cb_dt<8, true>(a, st) : launch_cb_dt<8, false>(a, st);
 }
 
 }  // namespace moe
