@@ -45,8 +45,12 @@ namespace moe {
 // plain copy
 // ------------------------------------------------------------------------------------------
 
-constexpr int DC_STAGES = 6;
-constexpr int DC_CHUNK = 4096;
+// A 12-stage ring of 2 KB chunks (24 KB per CTA, as the earlier 6 x 4 KB).  In
+// the graph-replayed step, three interleaved process pairs: 16384 x 2048 rows
+// 253.6 -> 252.3 us, 4096 x 768 40.9 -> 40.6 us, 1024 x 768 19.09 -> 18.85 us;
+// 8 x 4 KB and 4 x 4 KB landed in between, 6 x 2 KB was slower (260.6 us).
+constexpr int DC_STAGES = 12;
+constexpr int DC_CHUNK = 2048;
 
 struct CopyArgs {
     const uint8_t *x;
