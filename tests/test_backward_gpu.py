@@ -46,6 +46,8 @@ CASES = [
     synth.WORKLOADS["4"].replace(S=300, H=2304, dtype="f32"),  # fp32 rows of 9 KB
     synth.WORKLOADS["5"].replace(S=700, H=1536, dtype="f32"),  # fp32 rows of 6 KB: 6 warps, 3 KB chunks
     synth.Workload("bwd_ragged", 777, 264, 40, 5, 4, 3, "bf16", "none", True, seed=31),
+    synth.Workload("bwd_2k", 300, 1032, 40, 5, 4, 3, "bf16", "none", True, seed=33),   # 2064-byte rows: 6 warps
+    synth.Workload("bwd_8k", 200, 4104, 32, 4, 4, 0, "bf16", "none", True, seed=34),   # 8208-byte rows: 16 warps
     synth.Workload("bwd_k17_f32", 301, 260, 17, 17, 17, 1, "f32", "none", True, seed=32),
 ]
 

@@ -43,6 +43,9 @@ RAGGED = [
     _wl(5000, 64, 8, 2, 2, 0, "f32", "none", False, 17),
     _wl(77, 128, 32, 32, 4, 3, "bf16", "fp8", True, 18),
     _wl(4099, 264, 384, 8, 4, 128, "bf16", "none", False, 19),
+    _wl(700, 1032, 64, 8, 8, 0, "bf16", "none", True, 22),    # 2064-byte rows: just past 2 KB (6 combine warps)
+    _wl(333, 2048, 64, 6, 4, 16, "f32", "fp8", True, 23),     # 8 KB fp32 rows: three 3 KB chunks, FP8 dispatch
+    _wl(257, 4104, 32, 4, 4, 0, "bf16", "none", False, 24),   # 8208-byte rows: 8 warps, a 16-byte last chunk
 ]
 
 
